@@ -1,0 +1,420 @@
+"""Benchmark of the NVFP4 W4A4 linear hot path on B200.
+
+One step = the DiT QKV projection (X bf16 [2640, 3072], W bf16 [9216, 3072])
+through the whole path: global amax + 1D quantization of X (4-vs-6 on),
+global amax + 2D 16x16 quantization of W (4-vs-6 on), tcgen05 block-scaled
+FP4 GEMM Y = X W^T with a bf16 output.  `value` is whole-step throughput in
+TFLOP/s of the GEMM's 2*M*N*K (quantization time included), inputs resident
+in HBM, L2 flushed between steps, device-timed with CUDA events, max over
+ranks.  Each rank runs its own independent step (weak scaling, no data-path
+collective).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 GEMM TFLOPS (%FP4 peak) and quantize/dequant GB/s (%HBM) on 1 B200"
+M, N, K = 2640, 9216, 3072
+WORKLOAD = "DiT QKV projection W4A4: X bf16 [2640x3072] (1% Student-t(3)x8 channels), " \
+           "W bf16 [9216x3072] N(0,0.02); 1D act + 2D weight NVFP4, 4-vs-6 on; Y bf16 [2640x9216]"
+FLUSH_BYTES = 256 << 20
+# CPU-oracle sample: the first rows of the same workload
+CPU_MS, CPU_NS = 64, 128
+
+
+def peaks():
+    """Roofline denominators from MEASURED_PEAKS.json (driver-written), else
+    the pool's fallback measurement."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+        return self.summary()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ dist
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ CPU oracle
+def cpu_sample_step(x_rows, w_rows):
+    """The oracle on a bounded sample of the workload: quantize the first
+    CPU_MS activation rows and CPU_NS weight rows, then the fp64 GEMM of the
+    CPU_MS x CPU_NS outputs.  Returns the sample's 2*m*n*K."""
+    import oracle
+    a = oracle.quantize_1d(x_rows, sf_layout=oracle.SF_TCGEN05)
+    b = oracle.quantize_2d(w_rows, sf_layout=oracle.SF_TCGEN05)
+    oracle.gemm((a[0], a[1], a[2], 1), (b[0], b[1], b[2], 1), x_rows.shape[0], w_rows.shape[0], K)
+    return 2.0 * x_rows.shape[0] * w_rows.shape[0] * K
+
+
+def cpu_inputs():
+    from nvfp4_block_scaled_20_b200 import synth
+    x, w = synth.qkv_linear("cpu")
+    return (x[:CPU_MS].float().numpy().copy(), w[:CPU_NS].float().numpy().copy())
+
+
+def cpu_baseline(min_seconds=10.0):
+    import oracle
+    oracle.build()
+    xr, wr = cpu_inputs()
+    flops, t0, reps = 0.0, time.perf_counter(), 0
+    while True:
+        flops += cpu_sample_step(xr, wr)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    return {"value": flops / el / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": "%d reps of: 1D-quantize X[:%d], 2D-quantize W[:%d], fp64 GEMM %dx%dx%d "
+                      "(single-threaded C oracle)" % (reps, CPU_MS, CPU_NS, CPU_MS, CPU_NS, K)}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    xr, wr = cpu_inputs()
+    for _ in range(args.warmup):
+        cpu_sample_step(xr, wr)
+    t0 = time.perf_counter()
+    flops = 0.0
+    for _ in range(args.steps):
+        flops += cpu_sample_step(xr, wr)
+    el = time.perf_counter() - t0
+    v = flops / el / 1e12
+    sample = ("each step: 1D-quantize X[:%d], 2D-quantize W[:%d], fp64 GEMM %dx%dx%d "
+              "(single-threaded C oracle)" % (CPU_MS, CPU_NS, CPU_MS, CPU_NS, K))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32 encode / f64 accumulate", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": sample},
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    import torch
+    import nvfp4_block_scaled_20_b200 as nv
+    from nvfp4_block_scaled_20_b200 import build, synth
+    build.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    pk = peaks()
+
+    # inputs: each rank its own batch (seeded by rank), resident in HBM
+    x, w = synth.qkv_linear(dev)
+    if rank:
+        x = synth.activation(1 + 1000 * rank, 1, M, K, device=dev)
+        w = synth.weight(1 + 1000 * rank, 2, N, K, device=dev)
+    qa = nv.QTensor(*nv._alloc_q(M, K, nv.NVFP4_SF_TCGEN05, dev), M, K, nv.NVFP4_SF_TCGEN05)
+    qb = nv.QTensor(*nv._alloc_q(N, K, nv.NVFP4_SF_TCGEN05, dev), N, K, nv.NVFP4_SF_TCGEN05)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws_a, ws_b, ws_g = nv.workspace(1, dev), nv.workspace(1, dev), nv.workspace(0, dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def quant_x():
+        nv.quantize_1d(x, out=qa, ws=ws_a, stream=stream)
+
+    def quant_w():
+        nv.quantize_2d(w, out=qb, ws=ws_b, stream=stream)
+
+    def amax_x():
+        nv.global_scale(x, out=qa.alpha, ws=ws_a, stream=stream)
+
+    def pass2_x():
+        nv.quantize_1d(x, out=qa, ws=ws_a, alpha_in=qa.alpha, stream=stream)
+
+    def amax_w():
+        nv.global_scale(w, out=qb.alpha, ws=ws_b, stream=stream)
+
+    def pass2_w():
+        nv.quantize_2d(w, out=qb, ws=ws_b, alpha_in=qb.alpha, stream=stream)
+
+    def gemm():
+        nv.gemm(qa, qb, out=y, ws=ws_g, stream=stream)
+
+    def step():
+        quant_x()
+        quant_w()
+        gemm()
+
+    # warm-up (also sets kernel attributes before graph capture)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    assert nv.device_error(ws_g, stream) == 0
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        return g
+
+    graphs = {"step": capture(step), "amax_x": capture(amax_x), "pass2_x": capture(pass2_x),
+              "amax_w": capture(amax_w), "pass2_w": capture(pass2_w), "gemm": capture(gemm)}
+
+    def timed(g, reps):
+        """Mean device time (ms) of one graph replay, L2 flushed before each."""
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(2_000_000)  # let the host run ahead of the device
+            for s, e in evs:
+                flush.zero_()
+                s.record(stream)
+                g.replay()
+                e.record(stream)
+        stream.synchronize()
+        return sum(s.elapsed_time(e) for s, e in evs) / reps
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            graphs["step"].replay()
+    stream.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.2)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    step_ms = timed(graphs["step"], args.steps)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    # per-kernel breakdown (same protocol)
+    reps = max(20, min(args.steps, 200))
+    part = {k: timed(graphs[k], reps) for k in ("amax_x", "pass2_x", "amax_w", "pass2_w", "gemm")}
+    clk = clocks.stop()
+    assert nv.device_error(ws_g, stream) == 0
+
+    step_ms_max = reduce_max(step_ms, world, dev)
+    flops = 2.0 * M * N * K
+    value = world * flops / (step_ms_max * 1e-3) / 1e12
+
+    fp4_peak = 4.0 * pk["bf16_tflops"]  # nominal FP4:BF16 dense ratio 9 : 2.25
+    gemm_tflops = flops / (part["gemm"] * 1e-3) / 1e12
+    hbm = pk["hbm_gbs"]
+
+    def gbs(nbytes, ms):
+        v = nbytes / (ms * 1e-3) / 1e9
+        return {"ms": round(ms, 5), "GB/s": round(v, 1), "frac_hbm": round(v / hbm, 3)}
+
+    q_out = 0.5 + 1.0 / 16  # bytes written per element (codes + scale bytes)
+    breakdown = {
+        "gemm": {"ms": round(part["gemm"], 5), "TFLOP/s": round(gemm_tflops, 1),
+                 "frac_fp4_peak": round(gemm_tflops / fp4_peak, 3)},
+        "amax_x": gbs(2 * M * K, part["amax_x"]),
+        "quantize_x_pass2": gbs((2 + q_out) * M * K, part["pass2_x"]),
+        "amax_w": gbs(2 * N * K, part["amax_w"]),
+        "quantize_w_pass2": gbs((2 + q_out) * N * K, part["pass2_w"]),
+        "note": "inputs (X 16 MB, W 57 MB bf16) are smaller than L2; each kernel is timed after "
+                "an L2 flush, so a second pass over the same tensor inside one step may hit L2",
+    }
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(nv, torch, dev, stream, x, w, qa, qb, ws_a, ws_b, ws_g, args, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4 (e2m1 x e2m1, ue4m3 scales, fp32 accumulate; fp32 encode)",
+            "data": "synthetic (seeded splitmix64 generator, DiT QKV shapes)",
+            "config": {"workload": WORKLOAD, "M": M, "N": N, "K": K,
+                       "parallelism": "replica per GPU (weak scaling)" if world > 1 else "single GPU",
+                       "l2": "flushed: 256 MiB write before every timed step",
+                       "timing": "CUDA events around a CUDA-graph replay of the step, max over ranks"},
+            "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1),
+                         "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                         "frac": round(gemm_tflops / fp4_peak, 4), "traffic": None,
+                         "kernel": "gemm_kernel<256> (tcgen05.mma kind::mxf4nvf4)",
+                         "peak_source": "%s bf16 burst %.1f TFLOP/s x 4 (nominal dense FP4:BF16 "
+                                        "ratio)" % (pk["source"], pk["bf16_tflops"])},
+            "breakdown": breakdown,
+            "gpu_launches": 5 * args.steps,
+            "clocks": clk,
+        }
+        if e2e:
+            line["e2e"] = e2e
+        if cpu:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        del graphs
+        dist.destroy_process_group()
+    return 0
+
+
+def measure_e2e(nv, torch, dev, stream, x, w, qa, qb, ws_a, ws_b, ws_g, args, world):
+    """Same step through the public API with the inputs copied from pinned host
+    memory and the bf16 result copied back, every step."""
+    hx = x.cpu().pin_memory()
+    hw = w.cpu().pin_memory()
+    hy = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    dx = torch.empty_like(x)
+    dw = torch.empty_like(w)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    steps = max(3, min(args.steps, 50))
+
+    def one():
+        dx.copy_(hx, non_blocking=True)
+        dw.copy_(hw, non_blocking=True)
+        nv.quantize_1d(dx, out=qa, ws=ws_a, stream=stream)
+        nv.quantize_2d(dw, out=qb, ws=ws_b, stream=stream)
+        nv.gemm(qa, qb, out=y, ws=ws_g, stream=stream)
+        hy.copy_(y, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            one()
+    stream.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        s.record(stream)
+        for _ in range(steps):
+            one()
+        e.record(stream)
+    stream.synchronize()
+    ms = reduce_max(s.elapsed_time(e) / steps, world, dev)
+    return {"value": world * 2.0 * M * N * K / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": ms, "h2d_bytes_per_step": x.numel() * 2 + w.numel() * 2,
+            "d2h_bytes_per_step": M * N * 2}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

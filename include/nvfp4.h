@@ -1,0 +1,251 @@
+/*
+ * nvfp4.h -- C ABI of the B200 (sm_100a) NVFP4 W4A4 linear-layer library.
+ *
+ * NVFP4 as defined on the LongLive-2.0 pages ("LongLive-2.0: An NVFP4
+ * Parallel Infrastructure for Long Video Generation"; "explainer" below is
+ * the paper-graph-ui architecture page, section 3.4 "Detailed, Sentence-Based
+ * Technical Breakdown"):
+ *   X^ = X^_FP4 * a_FP8 * a_FP32  -- E2M1 4-bit elements, one FP8 E4M3 scale
+ *   per 16 elements, one FP32 scale per tensor ("NVFP4 numeric format",
+ *   "Hierarchical scaling").
+ *
+ * Conventions for every entry point
+ *   - Ownership: the caller allocates and frees every buffer (device memory
+ *     unless a parameter says "host").  The library never allocates, frees or
+ *     keeps a pointer after the call returns.
+ *   - Asynchrony: work is enqueued on `stream` (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream).  No call synchronizes, except
+ *     nvfp4_get_device_error.
+ *   - Errors: arguments are validated on the host before anything is
+ *     enqueued; a failed check returns a status and enqueues nothing.  A
+ *     CUDA launch failure returns NVFP4_ERR_CUDA.  Faults detected on the
+ *     device (a bounded wait that ran out) are recorded in the workspace
+ *     error word and read back with nvfp4_get_device_error.
+ *   - Element packing: two E2M1 codes per byte, element 2j in the low
+ *     nibble, element 2j+1 in the high nibble; code bit 3 is the sign.
+ *   - Scale bytes are UE4M3 (sign bit 0).  Two layouts:
+ *       NVFP4_SF_ROWMAJOR: byte (r, kb) at r * (cols/16) + kb.
+ *       NVFP4_SF_TCGEN05:  the tcgen05 block-scaled layout: 512-byte atoms of
+ *         128 rows x 4 blocks, byte (r, kb) at
+ *         ((r/128) * ceil(kb_total/4) + kb/4) * 512
+ *           + (r%32)*16 + ((r%128)/32)*4 + kb%4,
+ *         rows padded to a multiple of 128 and blocks to a multiple of 4;
+ *         the quantizers write zeros into the padding.
+ *   - Pointers to tensors must be 16-byte aligned; leading dimensions are in
+ *     elements and must keep every row 16-byte aligned.
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NVFP4_API __attribute__((visibility("default")))
+#else
+#define NVFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum nvfp4_status {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1, /* NULL pointer, unknown enum value            */
+  NVFP4_ERR_SHAPE = 2,       /* a dimension violates the call's shape rule  */
+  NVFP4_ERR_ALIGN = 3,       /* pointer or leading dimension misaligned     */
+  NVFP4_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than required     */
+  NVFP4_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed           */
+  NVFP4_ERR_TIMEOUT = 6,     /* a bounded device wait ran out (device side) */
+  NVFP4_ERR_UNSUPPORTED = 7  /* valid request this build does not implement */
+} nvfp4_status;
+
+typedef enum nvfp4_dtype { NVFP4_F32 = 0, NVFP4_BF16 = 1 } nvfp4_dtype;
+
+typedef enum nvfp4_sf_layout {
+  NVFP4_SF_ROWMAJOR = 0,
+  NVFP4_SF_TCGEN05 = 1
+} nvfp4_sf_layout;
+
+typedef enum nvfp4_epilogue {
+  NVFP4_EPI_NONE = 0,
+  NVFP4_EPI_GELU_TANH = 1 /* 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))) */
+} nvfp4_epilogue;
+
+/* Quantizer options.
+ *   four_over_six  1: per block, encode with the scale that maps the block
+ *                  max to 6 and with the one that maps it to 4, keep the one
+ *                  with the lower squared error (ties keep 6) -- explainer,
+ *                  NVFP4 Inference, "Scale-search mechanism".  0: 6-rule only
+ *                  ("Quantization rule for a tensor block").
+ *   rht_enable     1: 16-point random Hadamard transform of every 16-block
+ *                  (along the block axis) before amax and encoding --
+ *                  explainer, "Random Hadamard Transform (RHT) for gradient
+ *                  stabilization".  1D quantizers only.
+ *   rht_sign_mask  bit j set => sign s_j = -1 in y = 1/4 H16 diag(s) x
+ *                  (Sylvester-ordered H16).
+ *   block_axis     0: 16-blocks along the contiguous dim: codes [rows,
+ *                  cols/2], scales for rows x cols/16.  1 (1D only): blocks
+ *                  along rows, output transposed: codes [cols, rows/2],
+ *                  scales for cols x rows/16 (WGRAD operands, K = tokens).
+ *   sf_layout      nvfp4_sf_layout of the scale output.
+ *   global_scale_in  device pointer to a_FP32; NULL => computed as
+ *                  amax / (6 * 448) over the (transformed) tensor, 1.0 for an
+ *                  all-zero tensor. */
+typedef struct nvfp4_qparams {
+  int32_t four_over_six;
+  int32_t rht_enable;
+  uint32_t rht_sign_mask;
+  int32_t block_axis;
+  int32_t sf_layout;
+  int32_t reserved0;
+  const float* global_scale_in;
+} nvfp4_qparams;
+
+/* One tensor of a batched call (KV cache: one per layer and K/V).
+ *   quantize:   x [rows, ld] input (dtype of the call), codes/scales outputs,
+ *               global_scale = device float written with a_FP32.
+ *   dequantize: codes/scales inputs, global_scale = device float a_FP32 read,
+ *               out [rows, ld] output (dtype of the call); x unused. */
+typedef struct nvfp4_tensor_desc {
+  const void* x;
+  void* out;
+  uint8_t* codes;
+  uint8_t* scales;
+  float* global_scale;
+  int64_t rows;
+  int64_t cols;
+  int64_t ld;
+} nvfp4_tensor_desc;
+
+/* ------------------------------------------------------------ sizes ---- */
+
+/* Bytes of device workspace a call needs: a device error word plus one
+ * 4-byte amax slot per tensor (n_tensors = 1 for the single-tensor calls,
+ * 0 for nvfp4_gemm).  The library zeroes what it uses on `stream`. */
+NVFP4_API size_t nvfp4_workspace_bytes(int32_t n_tensors);
+
+/* Bytes of the packed codes of a [rows, cols] block-axis-0 encoding. */
+NVFP4_API int64_t nvfp4_codes_bytes(int64_t rows, int64_t cols);
+
+/* Bytes of the scale buffer for `rows` rows of `cols` elements. */
+NVFP4_API int64_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int32_t sf_layout);
+
+/* ------------------------------------------------------------ quantize -- */
+
+/* Global scale only (the amax pass): *global_scale_out = a_FP32 of x under
+ * qp (RHT and block_axis honoured; qp->global_scale_in ignored).
+ * explainer, "Hierarchical scaling" (tensor-wise FP32 scale).
+ * x: device [rows, ld] of dtype.  Shape rules as nvfp4_quantize_1d. */
+NVFP4_API nvfp4_status nvfp4_global_scale(const void* x, int32_t dtype, int64_t rows,
+                                int64_t cols, int64_t ld,
+                                const nvfp4_qparams* qp,
+                                float* global_scale_out, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/* 1D NVFP4 quantization -- explainer, "NVFP4 training recipe for AR
+ * training" (1D blocks of 16 along the reduction dimension) and
+ * "Quantization rule for a tensor block".
+ *   x        device [rows, ld] of dtype (NVFP4_F32 or NVFP4_BF16).
+ *   codes    device, nvfp4_codes_bytes of the output shape.
+ *   scales   device, nvfp4_scales_bytes of the output shape and layout.
+ *   global_scale_out  device float; receives a_FP32 (may equal
+ *            qp->global_scale_in).
+ * Shape: cols % 16 == 0; block_axis 1 also needs rows % 16 == 0.
+ * Runs the amax pass then the quantize pass (one pass with
+ * global_scale_in).  Workspace: nvfp4_workspace_bytes(1). */
+NVFP4_API nvfp4_status nvfp4_quantize_1d(const void* x, int32_t dtype, int64_t rows,
+                               int64_t cols, int64_t ld,
+                               const nvfp4_qparams* qp, uint8_t* codes,
+                               uint8_t* scales, float* global_scale_out,
+                               void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* 2D NVFP4 quantization of a weight [rows, cols] in 16x16 tiles, one scale
+ * per tile (written to the scale entries of the tile's 16 rows), the 4-vs-6
+ * pick on the tile's 256 values -- explainer, "NVFP4 training recipe for AR
+ * training" (2D block scaling, "e.g., 16x16").  rows % 16 == 0,
+ * cols % 16 == 0; rht_enable and block_axis must be 0.  Arguments as
+ * nvfp4_quantize_1d. */
+NVFP4_API nvfp4_status nvfp4_quantize_2d(const void* x, int32_t dtype, int64_t rows,
+                               int64_t cols, int64_t ld,
+                               const nvfp4_qparams* qp, uint8_t* codes,
+                               uint8_t* scales, float* global_scale_out,
+                               void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* Batched 1D quantization (KV cache): n tensors, each with its own a_FP32
+ * (one per layer and K/V), all of one dtype, one launch per pass --
+ * explainer, "KV cache quantization" / "Chunkwise quantization procedure"
+ * ([T*H, d] rows, 16-blocks along d).  qp applies to every tensor
+ * (global_scale_in must be NULL: each tensor gets its own scale).
+ * descs: HOST array of n descriptors.  Workspace: nvfp4_workspace_bytes(n). */
+NVFP4_API nvfp4_status nvfp4_quantize_1d_batched(const nvfp4_tensor_desc* descs,
+                                       int32_t n, int32_t dtype,
+                                       const nvfp4_qparams* qp,
+                                       void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------ dequant --- */
+
+/* Parallel dequantization of n tensors in one launch: out = val(q) * d *
+ * a_FP32 (fp32 product, then round-to-nearest-even to bf16 for NVFP4_BF16)
+ * -- explainer, "Hierarchical scaling" and "Parallel CUDA dequantization
+ * kernel" (every CTA independent, all tensors in a single launch).
+ * descs: HOST array; per tensor codes/scales/global_scale are read and out
+ * [rows, ld] of out_dtype is written.  cols % 16 == 0. */
+NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor_desc* descs, int32_t n,
+                              int32_t out_dtype, int32_t sf_layout,
+                              void* stream);
+
+/* ------------------------------------------------------------ GEMM ------ */
+
+/* Block-scaled FP4 GEMM on the 5th-generation tensor cores
+ * (tcgen05.mma kind::mxf4nvf4, UE4M3 scales per 16 elements, fp32
+ * accumulation in tensor memory):
+ *   out[m, n] = epi( a_alpha * b_alpha *
+ *                    sum_k val(a_mk) sA[m, k/16] * val(b_nk) sB[n, k/16] )
+ * -- explainer, "The three GEMMs of backpropagation in NVFP4" (Y = X W^T
+ * forward, WGRAD with both operands quantized along the tokens).
+ *   a_codes  device [M, K/2] (K-major),  a_sf device, NVFP4_SF_TCGEN05
+ *            layout for M rows, K/16 blocks;  a_alpha device float.
+ *   b_codes  device [N, K/2] (K-major),  b_sf, b_alpha likewise for N rows.
+ *   out      device [M, ldo] of out_dtype (NVFP4_BF16: RNE; NVFP4_F32).
+ *   epilogue nvfp4_epilogue, applied in fp32 before the conversion.
+ * Shape: M >= 1, N % 16 == 0, K % 64 == 0, ldo >= N, ldo * elem % 16 == 0.
+ * Workspace: nvfp4_workspace_bytes(0) (the device error word). */
+NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf,
+                        const float* a_alpha, const uint8_t* b_codes,
+                        const uint8_t* b_sf, const float* b_alpha, int64_t M,
+                        int64_t N, int64_t K, void* out, int32_t out_dtype,
+                        int64_t ldo, int32_t epilogue, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------ RHT ------- */
+
+/* Standalone 16-point RHT, y = 1/4 H16 diag(s) x on every 16-group along
+ * block_axis (0: contiguous dim, cols % 16 == 0; 1: rows, rows % 16 == 0),
+ * the same transform the quantizers fuse -- explainer, "Random Hadamard
+ * Transform (RHT) for gradient stabilization".
+ *   x device [rows, ld] of dtype; out device fp32 [rows, cols]. */
+NVFP4_API nvfp4_status nvfp4_rht16(const void* x, int32_t dtype, int64_t rows,
+                         int64_t cols, int64_t ld, int32_t block_axis,
+                         uint32_t sign_mask, float* out, void* stream);
+
+/* ------------------------------------------------------------ status ---- */
+
+/* Synchronizes `stream`, copies the workspace's device error word to the
+ * HOST int32 *error_out (0 = none, else an nvfp4_status value) and clears
+ * it.  Returns NVFP4_ERR_CUDA if the copy fails. */
+NVFP4_API nvfp4_status nvfp4_get_device_error(void* workspace, int32_t* error_out,
+                                    void* stream);
+
+/* Static, NUL-terminated description of a status value. */
+NVFP4_API const char* nvfp4_status_string(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

@@ -1,0 +1,287 @@
+// C ABI of the NVFP4 library (declared in include/nvfp4.h): argument
+// validation on the host, workspace carve-up, kernel launches.  Nothing here
+// allocates device memory or synchronizes (except nvfp4_get_device_error).
+#include <cstring>
+
+#include "../../include/nvfp4.h"
+#include "kernels.h"
+
+using namespace nvfp4;
+
+namespace {
+
+constexpr size_t kErrWordBytes = 256;  // error word, padded
+inline bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+inline int64_t elem_bytes(int32_t dt) { return dt == NVFP4_BF16 ? 2 : 4; }
+inline bool dtype_ok(int32_t dt) { return dt == NVFP4_F32 || dt == NVFP4_BF16; }
+inline cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
+
+uint32_t* err_word(void* ws) { return static_cast<uint32_t*>(ws); }
+uint32_t* amax_slots(void* ws) {
+  return reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + kErrWordBytes);
+}
+
+// Shape / alignment rules of one quantizer input.
+nvfp4_status check_input(const void* x, int32_t dtype, int64_t rows, int64_t cols, int64_t ld,
+                         int block_axis, bool two_d) {
+  if (!dtype_ok(dtype)) return NVFP4_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0 || ld < cols) return NVFP4_ERR_SHAPE;
+  if (!x && rows > 0 && cols > 0) return NVFP4_ERR_INVALID_ARG;
+  if (block_axis == 0 && cols % 16) return NVFP4_ERR_SHAPE;
+  if ((block_axis == 1 || two_d) && rows % 16) return NVFP4_ERR_SHAPE;
+  if (two_d && cols % 16) return NVFP4_ERR_SHAPE;
+  if (block_axis == 1 && cols % 8) return NVFP4_ERR_SHAPE;
+  // the kernels index blocks with 32-bit integers
+  if ((double)rows * (double)cols / 16.0 >= 4.0e9) return NVFP4_ERR_SHAPE;
+  // contiguous 16-blocks are read with 256-bit loads: 32-byte aligned rows;
+  // the row-axis path reads element pairs: 16-byte aligned rows suffice
+  const size_t need = (block_axis == 0 || two_d) ? 32 : 16;
+  if (!aligned(x, need) || (ld * elem_bytes(dtype)) % (int64_t)need) return NVFP4_ERR_ALIGN;
+  return NVFP4_OK;
+}
+
+nvfp4_status check_qparams(const nvfp4_qparams* qp, bool two_d) {
+  if (!qp) return NVFP4_ERR_INVALID_ARG;
+  if (qp->block_axis != 0 && qp->block_axis != 1) return NVFP4_ERR_INVALID_ARG;
+  if (qp->sf_layout != NVFP4_SF_ROWMAJOR && qp->sf_layout != NVFP4_SF_TCGEN05)
+    return NVFP4_ERR_INVALID_ARG;
+  if (two_d && (qp->rht_enable || qp->block_axis != 0)) return NVFP4_ERR_INVALID_ARG;
+  if (qp->global_scale_in && !aligned(qp->global_scale_in, 4)) return NVFP4_ERR_ALIGN;
+  return NVFP4_OK;
+}
+
+void fill_batch_common(QBatch& b, int32_t dtype, const nvfp4_qparams* qp, void* ws) {
+  std::memset(&b, 0, sizeof(b));
+  b.bf16 = dtype == NVFP4_BF16;
+  b.four_over_six = qp->four_over_six != 0;
+  b.rht = qp->rht_enable != 0;
+  b.mask = qp->rht_sign_mask;
+  b.block_axis = qp->block_axis;
+  b.sf_layout = qp->sf_layout;
+  b.gs_in = qp->global_scale_in;
+  b.amax_slots = ws ? amax_slots(ws) : nullptr;
+}
+
+nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+nvfp4_status quantize_common(const void* x, int32_t dtype, int64_t rows, int64_t cols, int64_t ld,
+                             const nvfp4_qparams* qp, uint8_t* codes, uint8_t* scales,
+                             float* gs_out, void* ws, size_t ws_bytes, void* stream, bool two_d) {
+  nvfp4_status st = check_qparams(qp, two_d);
+  if (st != NVFP4_OK) return st;
+  st = check_input(x, dtype, rows, cols, ld, qp->block_axis, two_d);
+  if (st != NVFP4_OK) return st;
+  if (rows == 0 || cols == 0) return NVFP4_OK;  // empty: nothing to read or write
+  if (!codes || !scales || !gs_out) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(scales, 4) || !aligned(gs_out, 4)) return NVFP4_ERR_ALIGN;
+  if (!ws || ws_bytes < nvfp4_workspace_bytes(1)) return NVFP4_ERR_WORKSPACE;
+  QBatch b;
+  fill_batch_common(b, dtype, qp, ws);
+  b.n = 1;
+  b.t[0] = QTensor{x, codes, scales, gs_out, rows, cols, ld};
+  if (!qp->global_scale_in) {
+    cudaError_t e = cudaMemsetAsync(amax_slots(ws), 0, sizeof(uint32_t), S(stream));
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    e = launch_amax(b, S(stream));
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  }
+  return cuda_status(two_d ? launch_quantize_2d(b, S(stream)) : launch_quantize_1d(b, S(stream)));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t nvfp4_workspace_bytes(int32_t n_tensors) {
+  if (n_tensors < 0) n_tensors = 0;
+  return kErrWordBytes + ((size_t)n_tensors * 4 + 255) / 256 * 256;
+}
+
+int64_t nvfp4_codes_bytes(int64_t rows, int64_t cols) { return rows * cols / 2; }
+
+int64_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int32_t sf_layout) {
+  const int64_t kb = cols / 16;
+  if (sf_layout == NVFP4_SF_TCGEN05) return (rows + 127) / 128 * 128 * ((kb + 3) / 4) * 4;
+  return rows * kb;
+}
+
+nvfp4_status nvfp4_global_scale(const void* x, int32_t dtype, int64_t rows, int64_t cols,
+                                int64_t ld, const nvfp4_qparams* qp, float* global_scale_out,
+                                void* ws, size_t ws_bytes, void* stream) {
+  nvfp4_status st = check_qparams(qp, false);
+  if (st != NVFP4_OK) return st;
+  st = check_input(x, dtype, rows, cols, ld, qp->block_axis, false);
+  if (st != NVFP4_OK) return st;
+  if (!global_scale_out) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(global_scale_out, 4)) return NVFP4_ERR_ALIGN;
+  if (!ws || ws_bytes < nvfp4_workspace_bytes(1)) return NVFP4_ERR_WORKSPACE;
+  QBatch b;
+  fill_batch_common(b, dtype, qp, ws);
+  b.gs_in = nullptr;
+  b.n = 1;
+  b.t[0] = QTensor{x, nullptr, nullptr, global_scale_out, rows, cols, ld};
+  cudaError_t e = cudaMemsetAsync(amax_slots(ws), 0, sizeof(uint32_t), S(stream));
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (rows > 0 && cols > 0) {
+    e = launch_amax(b, S(stream));
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  }
+  return cuda_status(launch_finalize_alpha(amax_slots(ws), global_scale_out, S(stream)));
+}
+
+nvfp4_status nvfp4_quantize_1d(const void* x, int32_t dtype, int64_t rows, int64_t cols,
+                               int64_t ld, const nvfp4_qparams* qp, uint8_t* codes,
+                               uint8_t* scales, float* global_scale_out, void* ws,
+                               size_t ws_bytes, void* stream) {
+  return quantize_common(x, dtype, rows, cols, ld, qp, codes, scales, global_scale_out, ws,
+                         ws_bytes, stream, false);
+}
+
+nvfp4_status nvfp4_quantize_2d(const void* x, int32_t dtype, int64_t rows, int64_t cols,
+                               int64_t ld, const nvfp4_qparams* qp, uint8_t* codes,
+                               uint8_t* scales, float* global_scale_out, void* ws,
+                               size_t ws_bytes, void* stream) {
+  return quantize_common(x, dtype, rows, cols, ld, qp, codes, scales, global_scale_out, ws,
+                         ws_bytes, stream, true);
+}
+
+nvfp4_status nvfp4_quantize_1d_batched(const nvfp4_tensor_desc* descs, int32_t n, int32_t dtype,
+                                       const nvfp4_qparams* qp, void* ws, size_t ws_bytes,
+                                       void* stream) {
+  if (!descs || n < 0) return NVFP4_ERR_INVALID_ARG;
+  nvfp4_status st = check_qparams(qp, false);
+  if (st != NVFP4_OK) return st;
+  if (qp->global_scale_in) return NVFP4_ERR_INVALID_ARG;
+  if (!dtype_ok(dtype)) return NVFP4_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < n; ++i) {
+    const nvfp4_tensor_desc& d = descs[i];
+    st = check_input(d.x, dtype, d.rows, d.cols, d.ld, qp->block_axis, false);
+    if (st != NVFP4_OK) return st;
+    if (!d.codes || !d.scales || !d.global_scale) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(d.codes, 16) || !aligned(d.scales, 4) || !aligned(d.global_scale, 4))
+      return NVFP4_ERR_ALIGN;
+  }
+  if (!ws || ws_bytes < nvfp4_workspace_bytes(n)) return NVFP4_ERR_WORKSPACE;
+  if (n == 0) return NVFP4_OK;
+  cudaError_t e = cudaMemsetAsync(amax_slots(ws), 0, sizeof(uint32_t) * (size_t)n, S(stream));
+  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  for (int32_t base = 0; base < n; base += kMaxBatch) {
+    QBatch b;
+    fill_batch_common(b, dtype, qp, ws);
+    b.amax_slots = amax_slots(ws) + base;
+    b.n = (n - base) < kMaxBatch ? (n - base) : kMaxBatch;
+    for (int32_t i = 0; i < b.n; ++i) {
+      const nvfp4_tensor_desc& d = descs[base + i];
+      b.t[i] = QTensor{d.x, d.codes, d.scales, d.global_scale, d.rows, d.cols, d.ld};
+    }
+    e = launch_amax(b, S(stream));
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    e = launch_quantize_1d(b, S(stream));
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  }
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_dequantize(const nvfp4_tensor_desc* descs, int32_t n, int32_t out_dtype,
+                              int32_t sf_layout, void* stream) {
+  if (!descs || n < 0 || !dtype_ok(out_dtype)) return NVFP4_ERR_INVALID_ARG;
+  if (sf_layout != NVFP4_SF_ROWMAJOR && sf_layout != NVFP4_SF_TCGEN05) return NVFP4_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < n; ++i) {
+    const nvfp4_tensor_desc& d = descs[i];
+    if (!d.codes || !d.scales || !d.global_scale || !d.out) return NVFP4_ERR_INVALID_ARG;
+    if (d.rows < 0 || d.cols < 0 || d.cols % 16 || d.ld < d.cols) return NVFP4_ERR_SHAPE;
+    if ((double)d.rows * (double)d.cols / 16.0 >= 4.0e9) return NVFP4_ERR_SHAPE;
+    if (!aligned(d.codes, 8) || !aligned(d.out, 32) || (d.ld * elem_bytes(out_dtype)) % 32)
+      return NVFP4_ERR_ALIGN;
+  }
+  for (int32_t base = 0; base < n; base += kMaxBatch) {
+    DQBatch b;
+    std::memset(&b, 0, sizeof(b));
+    b.out_bf16 = out_dtype == NVFP4_BF16;
+    b.sf_layout = sf_layout;
+    b.n = 0;
+    for (int32_t i = base; i < n && i < base + kMaxBatch; ++i) {
+      const nvfp4_tensor_desc& d = descs[i];
+      if (d.rows == 0 || d.cols == 0) continue;
+      b.t[b.n++] = DQTensor{d.codes, d.scales, d.global_scale, d.out, d.rows, d.cols, d.ld};
+    }
+    if (b.n == 0) continue;
+    cudaError_t e = launch_dequantize(b, S(stream));
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  }
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_alpha,
+                        const uint8_t* b_codes, const uint8_t* b_sf, const float* b_alpha,
+                        int64_t M, int64_t N, int64_t K, void* out, int32_t out_dtype, int64_t ldo,
+                        int32_t epilogue, void* ws, size_t ws_bytes, void* stream) {
+  if (!a_codes || !a_sf || !a_alpha || !b_codes || !b_sf || !b_alpha || !out)
+    return NVFP4_ERR_INVALID_ARG;
+  if (!dtype_ok(out_dtype)) return NVFP4_ERR_INVALID_ARG;
+  if (epilogue != NVFP4_EPI_NONE && epilogue != NVFP4_EPI_GELU_TANH) return NVFP4_ERR_INVALID_ARG;
+  if (M < 1 || N < 16 || K < 64 || N % 16 || K % 64 || ldo < N) return NVFP4_ERR_SHAPE;
+  if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_sf, 16) || !aligned(b_sf, 16) ||
+      !aligned(out, 16) || (ldo * elem_bytes(out_dtype)) % 16 || !aligned(a_alpha, 4) ||
+      !aligned(b_alpha, 4))
+    return NVFP4_ERR_ALIGN;
+  if (!ws || ws_bytes < nvfp4_workspace_bytes(0)) return NVFP4_ERR_WORKSPACE;
+  GemmArgs g;
+  g.a_codes = a_codes;
+  g.a_sf = a_sf;
+  g.a_alpha = a_alpha;
+  g.b_codes = b_codes;
+  g.b_sf = b_sf;
+  g.b_alpha = b_alpha;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.out = out;
+  g.out_bf16 = out_dtype == NVFP4_BF16;
+  g.ldo = ldo;
+  g.epilogue = epilogue;
+  g.err = err_word(ws);
+  bool unsupported = false;
+  int e = launch_gemm(g, S(stream), &unsupported);
+  if (unsupported) return NVFP4_ERR_UNSUPPORTED;
+  return e == 0 ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+nvfp4_status nvfp4_rht16(const void* x, int32_t dtype, int64_t rows, int64_t cols, int64_t ld,
+                         int32_t block_axis, uint32_t sign_mask, float* out, void* stream) {
+  if (!x || !out || !dtype_ok(dtype)) return NVFP4_ERR_INVALID_ARG;
+  if (block_axis != 0 && block_axis != 1) return NVFP4_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0 || ld < cols) return NVFP4_ERR_SHAPE;
+  if ((block_axis == 0 && cols % 16) || (block_axis == 1 && rows % 16)) return NVFP4_ERR_SHAPE;
+  if (!aligned(x, (size_t)elem_bytes(dtype)) || !aligned(out, 4)) return NVFP4_ERR_ALIGN;
+  if (rows == 0 || cols == 0) return NVFP4_OK;
+  return cuda_status(launch_rht16(x, dtype == NVFP4_BF16, rows, cols, ld, block_axis, sign_mask,
+                                  out, S(stream)));
+}
+
+nvfp4_status nvfp4_get_device_error(void* ws, int32_t* error_out, void* stream) {
+  if (!ws || !error_out) return NVFP4_ERR_INVALID_ARG;
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, S(stream)) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  *error_out = (int32_t)v;
+  if (v != 0 && cudaMemsetAsync(ws, 0, sizeof(v), S(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
+  return NVFP4_OK;
+}
+
+const char* nvfp4_status_string(int32_t s) {
+  switch (s) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_SHAPE: return "shape violates the call's rules";
+    case NVFP4_ERR_ALIGN: return "pointer or leading dimension misaligned";
+    case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+    case NVFP4_ERR_CUDA: return "CUDA call failed";
+    case NVFP4_ERR_TIMEOUT: return "bounded device wait timed out";
+    case NVFP4_ERR_UNSUPPORTED: return "unsupported by this build";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,448 @@
+// Block-scaled NVFP4 GEMM on the sm_100a 5th-generation tensor cores.
+//
+//   out[m, n] = epi(alpha_a * alpha_b * sum_k a_mk * sA[m, k/16] * b_nk * sB[n, k/16])
+//
+// A [M, K] and B [N, K] are packed E2M1 codes (K-major), sA / sB are UE4M3
+// scales in the tcgen05 block-scaled layout.  One CTA computes a 128 x BN
+// tile of the output:
+//   warp 0      TMA producer: codes with cp.async.bulk.tensor (128B swizzle),
+//               scale atoms with cp.async.bulk, into a STAGES-deep ring;
+//   warp 1      allocates tensor memory and issues, from one thread, the
+//               tcgen05.cp of the stage's scale atoms into tensor memory and
+//               the tcgen05.mma kind::mxf4nvf4 (block16 scales, K = 64 each);
+//               tcgen05.commit releases the smem stage;
+//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (one row per
+//               thread), x alpha_a*alpha_b, optional GELU(tanh), bf16 / fp32
+//               stores.
+// Every wait is bounded (wall clock through %globaltimer); on a timeout the
+// CTA records NVFP4_ERR_TIMEOUT in the device error word, drains what it
+// issued and frees its tensor memory before returning.
+#include <cuda.h>
+
+#include "device_common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+
+namespace {
+
+constexpr int BM = 128;           // rows per CTA tile (one TMEM lane per row)
+constexpr int BK = 256;           // K elements per stage = 128 bytes of codes per row
+constexpr int BK_BYTES = BK / 2;  // one 128-byte swizzle row
+constexpr int MMA_K = 64;         // K per tcgen05.mma (kind::mxf4nvf4)
+constexpr int kNumThreads = 192;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
+constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s when draining after an abort
+
+template <int BN>
+struct Cfg {
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kABytes = BM * BK_BYTES;               // 16 KB
+  static constexpr int kBBytes = BN * BK_BYTES;               // 16 / 32 KB
+  static constexpr int kSfaBytes = 4 * 512;                   // 4 atoms (128 rows x 16 blocks)
+  static constexpr int kSfbBytes = (BN / 128) * 4 * 512;
+  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+  static constexpr int kTmemCols = BN == 256 ? 512 : 256;     // accumulator + scale factors
+  static constexpr int kSfaCol = BN;                          // 4 MMAs x 4 columns
+  static constexpr int kSfbCol = BN + 16;                     // 4 MMAs x (BN/32) columns
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+// --------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait; returns false on timeout or when another role aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63) == 0) {
+      if (abort_flag && *abort_flag) return false;
+      if (globaltimer() - t0 > limit_ns) return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t c0,
+                                            int32_t c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(dst),
+      "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "p; }" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t r[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05 format): start address >> 4 in
+// bits 0-13, leading byte offset >> 4 in 16-29, stride byte offset >> 4 in
+// 32-45, version 1 in 46-47, base offset 0, layout type in 61-63.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
+  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+}
+// K-major operand tile, 128-byte swizzle: rows of 128 bytes, 8-row groups
+// 1024 bytes apart.
+__device__ __forceinline__ uint64_t operand_desc(uint32_t addr) {
+  return smem_desc(addr, 16, 1024, 2 /*SWIZZLE_128B*/);
+}
+// Scale atom source for tcgen05.cp 32x128b: 32 rows x 16 bytes, contiguous
+// (8-row core matrices 128 bytes apart, no swizzle).
+__device__ __forceinline__ uint64_t sf_desc(uint32_t addr) {
+  return smem_desc(addr, 0, 128, 0 /*SWIZZLE_NONE*/);
+}
+// Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (format 1), UE4M3
+// scales (bit 23 = 0), K-major A and B, N >> 3 in bits 17-22, M >> 4 in
+// bits 24-28, scale-factor ids 0.
+__host__ __device__ constexpr uint32_t instr_desc(int M, int N) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ float gelu_tanh(float y) {
+  const float k0 = 0.7978845608028654f, k1 = 0.044715f;
+  const float y3 = __fmul_rn(__fmul_rn(y, y), y);
+  const float inner = __fmul_rn(k0, __fadd_rn(y, __fmul_rn(k1, y3)));
+  return __fmul_rn(__fmul_rn(0.5f, y), __fadd_rn(1.0f, tanhf(inner)));
+}
+
+struct Params {
+  const uint8_t* a_sf;
+  const uint8_t* b_sf;
+  const float* a_alpha;
+  const float* b_alpha;
+  void* out;
+  int64_t ldo;
+  int32_t M, N, K;
+  int32_t out_bf16;
+  int32_t epilogue;
+  uint32_t* err;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(kNumThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ Params p) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + C::kStages * C::kABytes;
+  uint8_t* sSFA = sB + C::kStages * C::kBBytes;
+  uint8_t* sSFB = sSFA + C::kStages * C::kSfaBytes;
+  uint64_t* bars = (uint64_t*)(sSFB + C::kStages * C::kSfbBytes);
+  uint64_t* full = bars;                    // [kStages]
+  uint64_t* empty = bars + C::kStages;      // [kStages]
+  uint64_t* accum = bars + 2 * C::kStages;  // [1]
+  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * C::kStages + 1);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  const int num_kt = (p.K + BK - 1) / BK;
+  const int kgroups = p.K / 64;  // 4-block scale groups per row band
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    mbar_init(smem_u32(accum), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(C::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued = 0;
+      bool ok = true;
+      for (int kt = 0; kt < num_kt && ok; ++kt) {
+        const int s = kt % C::kStages;
+        const uint32_t round = (uint32_t)(kt / C::kStages);
+        if (!mbar_wait(smem_u32(&empty[s]), (round & 1u) ^ 1u, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        const int atoms = min(4, kgroups - kt * 4);
+        uint32_t bytes = C::kABytes + C::kBBytes + atoms * 512;
+        const int nbands_total = (p.N + 127) / 128;
+        int bands = 0;
+        for (int b = 0; b < BN / 128; ++b)
+          if (n0 / 128 + b < nbands_total) ++bands;
+        bytes += bands * atoms * 512;
+        const uint32_t fb = smem_u32(&full[s]);
+        mbar_expect_tx(fb, bytes);
+        tma_load_2d(smem_u32(sA + s * C::kABytes), &tmA, kt * BK_BYTES, m0, fb);
+        tma_load_2d(smem_u32(sB + s * C::kBBytes), &tmB, kt * BK_BYTES, n0, fb);
+        bulk_load(smem_u32(sSFA + s * C::kSfaBytes),
+                  p.a_sf + ((int64_t)(m0 / 128) * kgroups + kt * 4) * 512, atoms * 512, fb);
+        for (int b = 0; b < bands; ++b)
+          bulk_load(smem_u32(sSFB + s * C::kSfbBytes + b * 2048),
+                    p.b_sf + ((int64_t)(n0 / 128 + b) * kgroups + kt * 4) * 512, atoms * 512, fb);
+        issued = kt + 1;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(p.err, kDevErrTimeout);
+      }
+      // Drain: every stage this thread issued must have landed before the
+      // CTA can retire (bounded).
+      for (int kt = (issued > C::kStages ? issued - C::kStages : 0); kt < issued; ++kt) {
+        const int s = kt % C::kStages;
+        mbar_wait(smem_u32(&full[s]), (uint32_t)(kt / C::kStages) & 1u, nullptr, kDrainLimitNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc(BM, BN);
+      const uint32_t t_acc = tmem;
+      const uint32_t t_sfa = tmem + C::kSfaCol;
+      const uint32_t t_sfb = tmem + C::kSfbCol;
+      bool ok = true;
+      for (int kt = 0; kt < num_kt; ++kt) {
+        const int s = kt % C::kStages;
+        if (!mbar_wait(smem_u32(&full[s]), (uint32_t)(kt / C::kStages) & 1u, abort_flag,
+                       kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int nmma = min(4, (p.K - kt * BK) / MMA_K);
+        const uint32_t a_base = smem_u32(sA + s * C::kABytes);
+        const uint32_t b_base = smem_u32(sB + s * C::kBBytes);
+        const uint32_t sfa_base = smem_u32(sSFA + s * C::kSfaBytes);
+        const uint32_t sfb_base = smem_u32(sSFB + s * C::kSfbBytes);
+        for (int k = 0; k < nmma; ++k) {
+          tc_cp_sf(t_sfa + 4 * k, sf_desc(sfa_base + 512 * k));
+#pragma unroll
+          for (int b = 0; b < BN / 128; ++b)
+            tc_cp_sf(t_sfb + (BN / 32) * k + 4 * b, sf_desc(sfb_base + 2048 * b + 512 * k));
+        }
+        for (int k = 0; k < nmma; ++k) {
+          tc_mma(t_acc, operand_desc(a_base + 32 * k), operand_desc(b_base + 32 * k), idesc,
+                 t_sfa + 4 * k, t_sfb + (BN / 32) * k, (kt > 0 || k > 0) ? 1u : 0u);
+        }
+        tc_commit(smem_u32(&empty[s]));
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        atomicOr(p.err, kDevErrTimeout);
+      }
+      // Always signal the accumulator barrier: it completes once every
+      // tcgen05 operation issued above has finished.
+      tc_commit(smem_u32(accum));
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
+    const bool ok = mbar_wait(smem_u32(accum), 0, nullptr, kWaitLimitNs);
+    tc_fence_after();
+    if (ok && !*abort_flag) {
+      const float scale = __fmul_rn(*p.a_alpha, *p.b_alpha);
+      const int row = m0 + quad * 32 + lane;
+      const bool row_ok = row < p.M;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, r);
+        const int col = n0 + c0;
+        if (!row_ok || col >= p.N) continue;
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          v[i] = __fmul_rn(__uint_as_float(r[i]), scale);
+          if (p.epilogue == 1) v[i] = gelu_tanh(v[i]);
+        }
+        if (p.out_bf16) {
+          uint32_t w[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t*>(&h);
+          }
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + (int64_t)row * p.ldo + col;
+          uint4* d4 = reinterpret_cast<uint4*>(dst);
+          d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        } else {
+          float* dst = static_cast<float*>(p.out) + (int64_t)row * p.ldo + col;
+          float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+      }
+    } else if (!ok) {
+      atomicOr(p.err, kDevErrTimeout);
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    // the accumulator barrier (bounded) guarantees no tcgen05 op is in flight
+    mbar_wait(smem_u32(accum), 0, nullptr, kDrainLimitNs);
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(C::kTmemCols)
+                 : "memory");
+  }
+}
+
+// --------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)ptr;
+  }
+  return fn;
+}
+
+// Codes [rows, K/2] bytes, box = 128 bytes x box_rows rows, 128-byte swizzle,
+// out-of-bounds rows / columns read as zero.
+bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+  cuuint32_t box[2] = {(cuuint32_t)BK_BYTES, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void*)codes, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN>
+int launch_bn(const GemmArgs& a, cudaStream_t s) {
+  using C = Cfg<BN>;
+  CUtensorMap tmA, tmB;
+  if (!make_codes_map(&tmA, a.a_codes, a.M, a.K, BM)) return (int)cudaErrorInvalidValue;
+  if (!make_codes_map(&tmB, a.b_codes, a.N, a.K, BN)) return (int)cudaErrorInvalidValue;
+  Params p;
+  p.a_sf = a.a_sf;
+  p.b_sf = a.b_sf;
+  p.a_alpha = a.a_alpha;
+  p.b_alpha = a.b_alpha;
+  p.out = a.out;
+  p.ldo = a.ldo;
+  p.M = (int32_t)a.M;
+  p.N = (int32_t)a.N;
+  p.K = (int32_t)a.K;
+  p.out_bf16 = a.out_bf16;
+  p.epilogue = a.epilogue;
+  p.err = a.err;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return (int)e;
+    attr_set = true;
+  }
+  dim3 grid((unsigned)((a.N + BN - 1) / BN), (unsigned)((a.M + BM - 1) / BM));
+  gemm_kernel<BN><<<grid, kNumThreads, C::kSmemBytes, s>>>(tmA, tmB, p);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace
+
+int launch_gemm(const GemmArgs& a, cudaStream_t s, bool* unsupported) {
+  *unsupported = false;
+  if (a.M > (int64_t)INT32_MAX / 2 || a.N > (int64_t)INT32_MAX / 2 || a.K > (int64_t)INT32_MAX / 2) {
+    *unsupported = true;
+    return 0;
+  }
+  if (a.N <= 128) return launch_bn<128>(a, s);
+  return launch_bn<256>(a, s);
+}
+
+}  // namespace nvfp4

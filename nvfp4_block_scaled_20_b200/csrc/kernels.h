@@ -1,0 +1,80 @@
+// Internal launcher interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nvfp4 {
+
+constexpr int kMaxBatch = 64;  // tensors per batched launch (kernel parameter space)
+
+struct QTensor {
+  const void* x;
+  uint8_t* codes;
+  uint8_t* scales;
+  float* gs_out;
+  int64_t rows;  // input rows
+  int64_t cols;  // input cols
+  int64_t ld;    // input leading dimension (elements)
+};
+
+struct QBatch {
+  QTensor t[kMaxBatch];
+  int32_t n;
+  int32_t bf16;  // 1: bf16 input, 0: fp32
+  int32_t four_over_six;
+  int32_t rht;
+  uint32_t mask;
+  int32_t block_axis;
+  int32_t sf_layout;
+  const float* gs_in;   // device; nullptr => from amax slots
+  uint32_t* amax_slots; // device, one per tensor (float bits), zeroed by the caller
+};
+
+struct DQTensor {
+  const uint8_t* codes;
+  const uint8_t* scales;
+  const float* gs;
+  void* out;
+  int64_t rows, cols, ldo;
+};
+
+struct DQBatch {
+  DQTensor t[kMaxBatch];
+  int32_t n;
+  int32_t out_bf16;
+  int32_t sf_layout;
+};
+
+struct GemmArgs {
+  const uint8_t* a_codes;
+  const uint8_t* a_sf;
+  const float* a_alpha;
+  const uint8_t* b_codes;
+  const uint8_t* b_sf;
+  const float* b_alpha;
+  int64_t M, N, K;
+  void* out;
+  int32_t out_bf16;
+  int64_t ldo;
+  int32_t epilogue;
+  uint32_t* err;  // device error word
+};
+
+int num_sms();
+
+// Each returns a cudaError_t from the launch.
+cudaError_t launch_amax(const QBatch& b, cudaStream_t s);
+cudaError_t launch_quantize_1d(const QBatch& b, cudaStream_t s);
+cudaError_t launch_quantize_2d(const QBatch& b, cudaStream_t s);
+cudaError_t launch_dequantize(const DQBatch& b, cudaStream_t s);
+cudaError_t launch_rht16(const void* x, int bf16, int64_t rows, int64_t cols, int64_t ld,
+                         int block_axis, uint32_t mask, float* out, cudaStream_t s);
+// Writes a_FP32 from the amax slot of tensor 0 to gs_out (amax-only call).
+cudaError_t launch_finalize_alpha(const uint32_t* amax_slot, float* gs_out, cudaStream_t s);
+// Returns 0 on success, a cudaError_t value otherwise; sets *unsupported for
+// shapes this build does not handle.
+int launch_gemm(const GemmArgs& a, cudaStream_t s, bool* unsupported);
+
+}  // namespace nvfp4

@@ -1,0 +1,121 @@
+"""C-ABI library: loads, exports every symbol include/nvfp4.h declares, and
+the host-side rules (sizes, validation) hold.  No compute call is made: every
+call here returns during host-side validation, before any CUDA work."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+from nvfp4_block_scaled_20_b200 import build, capi
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return capi.load()
+
+
+def declared_symbols():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            src = open(os.path.join(inc, f)).read()
+            names |= set(re.findall(r"NVFP4_API\s+[\w\s\*]*?\b(nvfp4_\w+)\s*\(", src))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert names == set(capi.EXPORTED)
+
+
+def test_size_helpers(lib):
+    assert capi.nvfp4_codes_bytes(2640, 3072) == 2640 * 1536
+    assert capi.nvfp4_scales_bytes(2640, 3072, capi.NVFP4_SF_ROWMAJOR) == 2640 * 192
+    # tcgen05 layout pads rows to 128 and blocks to 4
+    assert capi.nvfp4_scales_bytes(2640, 3072, capi.NVFP4_SF_TCGEN05) == 2688 * 192
+    assert capi.nvfp4_scales_bytes(64, 80, capi.NVFP4_SF_TCGEN05) == 128 * 8
+    assert capi.nvfp4_workspace_bytes(0) >= 4
+    assert capi.nvfp4_workspace_bytes(60) >= capi.nvfp4_workspace_bytes(0) + 240
+
+
+def test_status_strings(lib):
+    assert capi.nvfp4_status_string(0) == "ok"
+    for s in range(1, 8):
+        assert capi.nvfp4_status_string(s) != "unknown status"
+
+
+def _qp(**kw):
+    d = dict(four_over_six=1, rht_enable=0, rht_sign_mask=0, block_axis=0, sf_layout=1,
+             reserved0=0, global_scale_in=None)
+    d.update(kw)
+    return capi.nvfp4_qparams(**d)
+
+
+A = 1 << 20  # a fake, well-aligned address: never dereferenced (validation fails first)
+
+
+def test_quantize_validation(lib):
+    ws = capi.nvfp4_workspace_bytes(1)
+    q = capi.nvfp4_quantize_1d
+    # NULL input
+    assert q(None, 1, 64, 256, 256, _qp(), A, A, A, A, ws, None) == 1
+    # cols not a multiple of 16
+    assert q(A, 1, 64, 250, 250, _qp(), A, A, A, A, ws, None) == 2
+    # misaligned input / leading dimension
+    assert q(A + 2, 1, 64, 256, 256, _qp(), A, A, A, A, ws, None) == 3
+    assert q(A, 1, 64, 256, 264, _qp(), A, A, A, A, ws, None) == 3
+    # transposed path needs rows % 16
+    assert q(A, 1, 60, 256, 256, _qp(block_axis=1), A, A, A, A, ws, None) == 2
+    # workspace too small
+    assert q(A, 1, 64, 256, 256, _qp(), A, A, A, A, 0, None) == 4
+    # bad enum values
+    assert q(A, 7, 64, 256, 256, _qp(), A, A, A, A, ws, None) == 1
+    assert q(A, 1, 64, 256, 256, _qp(sf_layout=3), A, A, A, A, ws, None) == 1
+    # 2D: RHT not allowed, rows % 16
+    q2 = capi.nvfp4_quantize_2d
+    assert q2(A, 1, 64, 256, 256, _qp(rht_enable=1), A, A, A, A, ws, None) == 1
+    assert q2(A, 1, 40, 256, 256, _qp(), A, A, A, A, ws, None) == 2
+
+
+def test_gemm_validation(lib):
+    ws = capi.nvfp4_workspace_bytes(0)
+    g = capi.nvfp4_gemm
+    args = lambda M, N, K, ldo, out_dtype=1, epi=0, wsb=ws, a=A: (
+        a, A, A, A, A, A, M, N, K, A, out_dtype, ldo, epi, A, wsb, None)
+    assert g(*args(64, 128, 250, 128)) == 2      # K % 64
+    assert g(*args(64, 120, 256, 120)) == 2      # N % 16
+    assert g(*args(64, 128, 256, 100)) == 2      # ldo < N
+    assert g(*args(64, 128, 256, 136, 0)) == 3 or g(*args(64, 128, 256, 132, 1)) == 3
+    assert g(*args(64, 128, 256, 128, 5)) == 1   # dtype
+    assert g(*args(64, 128, 256, 128, 1, 9)) == 1  # epilogue
+    assert g(*args(64, 128, 256, 128, 1, 0, 0)) == 4  # workspace
+    assert g(*args(64, 128, 256, 128, 1, 0, ws, A + 8)) == 3  # misaligned codes
+    assert g(None, A, A, A, A, A, 64, 128, 256, A, 1, 128, 0, A, ws, None) == 1
+
+
+def test_batched_and_dequant_validation(lib):
+    d = (capi.nvfp4_tensor_desc * 2)()
+    d[0] = capi.nvfp4_tensor_desc(A, None, A, A, A, 64, 128, 128)
+    d[1] = capi.nvfp4_tensor_desc(A, None, A, A, A, 64, 120, 120)
+    ws = capi.nvfp4_workspace_bytes(2)
+    assert capi.nvfp4_quantize_1d_batched(d, 2, 1, _qp(), A, ws, None) == 2
+    assert capi.nvfp4_quantize_1d_batched(d, 1, 1, _qp(global_scale_in=A), A, ws, None) == 1
+    assert capi.nvfp4_quantize_1d_batched(d, 1, 1, _qp(), A, 4, None) == 4
+    e = (capi.nvfp4_tensor_desc * 1)()
+    e[0] = capi.nvfp4_tensor_desc(None, A, A, A, A, 64, 120, 128)
+    assert capi.nvfp4_dequantize(e, 1, 1, 0, None) == 2
+    e[0] = capi.nvfp4_tensor_desc(None, None, A, A, A, 64, 128, 128)
+    assert capi.nvfp4_dequantize(e, 1, 1, 0, None) == 1
+
+
+def test_rht_validation(lib):
+    assert capi.nvfp4_rht16(A, 1, 64, 100, 100, 0, 0, A, None) == 2
+    assert capi.nvfp4_rht16(A, 1, 60, 64, 64, 1, 0, A, None) == 2
+    assert capi.nvfp4_rht16(A, 1, 64, 64, 64, 2, 0, A, None) == 1

@@ -1,0 +1,121 @@
+"""GPU parity of the tcgen05 block-scaled FP4 GEMM against the oracle's fp64
+GEMM on the same encodings: |gpu - oracle| <= 1e-3 * sum_k |a_k b_k| (plus
+half a bf16 ulp of the reference for bf16 outputs), on shapes that span
+several tiles, ragged M / N tails, partial K stages and both tile widths."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import nvfp4_block_scaled_20_b200 as nv
+from nvfp4_block_scaled_20_b200 import synth
+from gpu_helpers import (DEV, assert_q_equal, gemm_tolerance, oracle_gemm_ref, require_gpu,
+                         to_oracle)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def upload(ref, rows, cols):
+    """Oracle encoding -> device QTensor (tcgen05 scale layout)."""
+    codes, scales, alpha = ref
+    return nv.QTensor(torch.from_numpy(codes).to(DEV), torch.from_numpy(scales).to(DEV),
+                      torch.tensor([alpha], dtype=torch.float32, device=DEV), rows, cols,
+                      nv.NVFP4_SF_TCGEN05)
+
+
+def run_case(x, w, out_dtype, epilogue=nv.NVFP4_EPI_NONE, x2d=False):
+    M, K = x.shape
+    N = w.shape[0]
+    aref = (oracle.quantize_2d if x2d else oracle.quantize_1d)(to_oracle(x), sf_layout=oracle.SF_TCGEN05)
+    bref = oracle.quantize_2d(to_oracle(w), sf_layout=oracle.SF_TCGEN05)
+    ws = nv.workspace(0)
+    out = nv.gemm(upload(aref, M, K), upload(bref, N, K), out_dtype=out_dtype, epilogue=epilogue,
+                  ws=ws)
+    assert nv.device_error(ws) == 0
+    y, s = oracle_gemm_ref(aref, bref, M, N, K)
+    if epilogue == nv.NVFP4_EPI_GELU_TANH:
+        y = np.vectorize(oracle.gelu_tanh)(y)
+    got = out.float().cpu().numpy().astype(np.float64)
+    tol = gemm_tolerance(y, s, out_dtype == torch.bfloat16, epilogue == nv.NVFP4_EPI_GELU_TANH)
+    err = np.abs(got - y)
+    bad = np.argwhere(err > tol)
+    assert bad.size == 0, "%d outputs out of tolerance, first %s: gpu=%r ref=%r tol=%r" % (
+        len(bad), bad[0], got[tuple(bad[0])], y[tuple(bad[0])], tol[tuple(bad[0])])
+    return got, y, s
+
+
+def test_tiny_linear_fp32_and_bf16():
+    x, w = synth.tiny_linear()  # M=64, N=128, K=256: one tile, BN=128 path
+    for dt in (torch.float32, torch.bfloat16):
+        run_case(x, w, dt)
+
+
+@pytest.mark.parametrize("M,N,K", [(200, 272, 320), (128, 256, 4096), (300, 384, 576),
+                                   (64, 128, 64), (1, 16, 256), (257, 512, 3072)])
+def test_shapes_bf16_inputs(M, N, K):
+    x = synth.activation(9, M + N, M, K)
+    w = synth.weight(9, K, N, K)
+    run_case(x, w, torch.float32)
+    run_case(x, w, torch.bfloat16)
+
+
+def test_gelu_epilogue():
+    x = synth.activation(10, 1, 130, 512)
+    w = synth.weight(10, 2, 256, 512)
+    run_case(x, w, torch.bfloat16, nv.NVFP4_EPI_GELU_TANH)
+    run_case(x, w, torch.float32, nv.NVFP4_EPI_GELU_TANH)
+
+
+def test_gpu_quantized_operands_end_to_end():
+    """The quantizers' device outputs fed straight into the GEMM (the product
+    path), codes checked bit-exact and the product within tolerance."""
+    x = synth.activation(11, 1, 192, 768)
+    w = synth.weight(11, 2, 320, 768)
+    qa = nv.quantize_1d(x.to(DEV))
+    qb = nv.quantize_2d(w.to(DEV))
+    aref = oracle.quantize_1d(to_oracle(x), sf_layout=1)
+    bref = oracle.quantize_2d(to_oracle(w), sf_layout=1)
+    assert_q_equal(qa, aref, "A")
+    assert_q_equal(qb, bref, "B")
+    out = nv.gemm(qa, qb, out_dtype=torch.float32).cpu().numpy()
+    y, s = oracle_gemm_ref(aref, bref, 192, 320, 768)
+    assert (np.abs(out - y) <= gemm_tolerance(y, s, False)).all()
+
+
+def test_wgrad_shape_transposed_operands():
+    """dW = dY^T X with both operands RHT-transformed and quantized along the
+    tokens (K), fp32 output."""
+    mask = synth.rht_sign_mask(0)
+    dy = synth.activation(4, 1, 1024, 128, n_out=0, std=1e-3)
+    x = synth.activation(4, 2, 1024, 272)
+    qa = nv.quantize_1d(dy.to(DEV), rht=True, mask=mask, block_axis=1)
+    qb = nv.quantize_1d(x.to(DEV), rht=True, mask=mask, block_axis=1)
+    aref = oracle.quantize_1d(to_oracle(dy), rht=True, mask=mask, block_axis=1, sf_layout=1)
+    bref = oracle.quantize_1d(to_oracle(x), rht=True, mask=mask, block_axis=1, sf_layout=1)
+    assert_q_equal(qa, aref, "dY^T")
+    assert_q_equal(qb, bref, "X^T")
+    out = nv.gemm(qa, qb, out_dtype=torch.float32).cpu().numpy()
+    y, s = oracle_gemm_ref(aref, bref, 128, 272, 1024)
+    assert (np.abs(out - y) <= gemm_tolerance(y, s, False)).all()
+    # and the transform-then-quantize product approximates the plain dY^T X
+    plain = to_oracle(dy).astype(np.float64).T @ to_oracle(x).astype(np.float64)
+    rel = np.linalg.norm(out - plain) / np.linalg.norm(plain)
+    assert rel < 0.2
+
+
+def test_ldo_larger_than_n():
+    x = synth.activation(12, 1, 96, 256)
+    w = synth.weight(12, 2, 144, 256)
+    aref = oracle.quantize_1d(to_oracle(x), sf_layout=1)
+    bref = oracle.quantize_2d(to_oracle(w), sf_layout=1)
+    big = torch.full((96, 200), -7.0, device=DEV)
+    nv.gemm(upload(aref, 96, 256), upload(bref, 144, 256), out=big[:, :144])
+    y, s = oracle_gemm_ref(aref, bref, 96, 144, 256)
+    got = big.cpu().numpy()
+    assert (np.abs(got[:, :144] - y) <= gemm_tolerance(y, s, False)).all()
+    assert (got[:, 144:] == -7.0).all()  # untouched
