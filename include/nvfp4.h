@@ -187,6 +187,25 @@ NVFP4_API nvfp4_status nvfp4_quantize_1d_batched(const nvfp4_tensor_desc* descs,
                                        void* workspace,
                                        size_t workspace_bytes, void* stream);
 
+/* Batched 1D quantization that takes no workspace (the paper has no
+ * counterpart; this is a library convenience).  For callers that cannot
+ * allocate device memory or pass a workspace: code running inside another
+ * framework's allocator that forbids side allocations, loops that must not
+ * call cudaMalloc because it synchronizes the device, or C callers holding
+ * only their tensors' raw pointers.  The per-tensor amax scratch is a fixed
+ * array inside the library (1 KB on every GPU that loads it, kept until the
+ * process exits); the call allocates and frees nothing.
+ *   descs, n, dtype, qp: as nvfp4_quantize_1d_batched; block_axis must be 0
+ *   and global_scale_in NULL.  n <= 256, else NVFP4_ERR_SHAPE.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Calls share the array: it keeps the last call's contents (each
+ * call clears the slots it uses), and calls that overlap on the GPU (other
+ * streams, other threads) race on it -- serialize them. */
+NVFP4_API nvfp4_status nvfp4_quantize_1d_batched_noalloc(const nvfp4_tensor_desc* descs,
+                                                         int32_t n, int32_t dtype,
+                                                         const nvfp4_qparams* qp, void* stream);
+
 /* ------------------------------------------------------------ dequant --- */
 
 /* Parallel dequantization of n tensors in one launch: out = val(q) * d *

@@ -21,7 +21,8 @@ NVFP4_EPI_NONE, NVFP4_EPI_GELU_TANH = 0, 1
 
 EXPORTED = [
     "nvfp4_workspace_bytes", "nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_global_scale",
-    "nvfp4_quantize_1d", "nvfp4_quantize_2d", "nvfp4_quantize_1d_batched", "nvfp4_dequantize",
+    "nvfp4_quantize_1d", "nvfp4_quantize_2d", "nvfp4_quantize_1d_batched",
+    "nvfp4_quantize_1d_batched_noalloc", "nvfp4_dequantize",
     "nvfp4_gemm", "nvfp4_rht16", "nvfp4_get_device_error", "nvfp4_status_string",
 ]
 
@@ -59,6 +60,7 @@ _SIGS = {
     "nvfp4_quantize_1d": (_I32, [_V, _I32, _I64, _I64, _I64, _QP, _V, _V, _V, _V, _SZ, _V]),
     "nvfp4_quantize_2d": (_I32, [_V, _I32, _I64, _I64, _I64, _QP, _V, _V, _V, _V, _SZ, _V]),
     "nvfp4_quantize_1d_batched": (_I32, [_TD, _I32, _I32, _QP, _V, _SZ, _V]),
+    "nvfp4_quantize_1d_batched_noalloc": (_I32, [_TD, _I32, _I32, _QP, _V]),
     "nvfp4_dequantize": (_I32, [_TD, _I32, _I32, _I32, _V]),
     "nvfp4_gemm": (_I32, [_V, _V, _V, _V, _V, _V, _I64, _I64, _I64, _V, _I32, _I64, _I32, _V,
                           _SZ, _V]),
@@ -123,6 +125,11 @@ def nvfp4_quantize_2d(x, dtype, rows, cols, ld, qp, codes, scales, gs_out, ws, w
 def nvfp4_quantize_1d_batched(descs, n, dtype, qp, ws, ws_bytes, stream):
     return _call("nvfp4_quantize_1d_batched", descs, n, dtype, ctypes.byref(qp), ws, ws_bytes,
                  stream)
+
+
+def nvfp4_quantize_1d_batched_noalloc(descs, n, dtype, qp, stream):
+    """Batched quantization with the library's own fixed scratch (no workspace)."""
+    return _call("nvfp4_quantize_1d_batched_noalloc", descs, n, dtype, ctypes.byref(qp), stream)
 
 
 def nvfp4_dequantize(descs, n, out_dtype, sf_layout, stream):
