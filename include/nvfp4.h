@@ -121,9 +121,11 @@ typedef struct nvfp4_tensor_desc {
 
 /* ------------------------------------------------------------ sizes ---- */
 
-/* Bytes of device workspace a call needs: a device error word plus one
- * 4-byte amax slot per tensor (n_tensors = 1 for the single-tensor calls,
- * 0 for nvfp4_gemm).  The library zeroes what it uses on `stream`. */
+/* Bytes of device workspace a call needs: a device error word plus the amax
+ * pass's per-CTA partial maxima for each tensor (n_tensors = 1 for the
+ * single-tensor calls, 0 for nvfp4_gemm).  Its contents need no
+ * initialization except the error word, which must start at zero (it is
+ * cleared by nvfp4_get_device_error). */
 NVFP4_API size_t nvfp4_workspace_bytes(int32_t n_tensors);
 
 /* Bytes of the packed codes of a [rows, cols] block-axis-0 encoding. */
@@ -193,15 +195,16 @@ NVFP4_API nvfp4_status nvfp4_quantize_1d_batched(const nvfp4_tensor_desc* descs,
  * framework's allocator that forbids side allocations, loops that must not
  * call cudaMalloc because it synchronizes the device, or C callers holding
  * only their tensors' raw pointers.  The per-tensor amax scratch is a fixed
- * array inside the library (1 KB on every GPU that loads it, kept until the
- * process exits); the call allocates and frees nothing.
+ * array inside the library (about 80 KB on every GPU that loads it, kept
+ * until the process exits); the call allocates and frees nothing.
  *   descs, n, dtype, qp: as nvfp4_quantize_1d_batched; block_axis must be 0
- *   and global_scale_in NULL.  n <= 256, else NVFP4_ERR_SHAPE.
+ *   and global_scale_in NULL.  n <= 64, else NVFP4_ERR_SHAPE.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
  * capture.  Calls share the array: it keeps the last call's contents (each
- * call clears the slots it uses), and calls that overlap on the GPU (other
- * streams, other threads) race on it -- serialize them. */
+ * call overwrites every slot it reads before reading it), and calls that
+ * overlap on the GPU (other streams, other threads) race on it -- serialize
+ * them. */
 NVFP4_API nvfp4_status nvfp4_quantize_1d_batched_noalloc(const nvfp4_tensor_desc* descs,
                                                          int32_t n, int32_t dtype,
                                                          const nvfp4_qparams* qp, void* stream);

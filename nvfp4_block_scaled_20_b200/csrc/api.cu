@@ -16,9 +16,11 @@ inline int64_t elem_bytes(int32_t dt) { return dt == NVFP4_BF16 ? 2 : 4; }
 inline bool dtype_ok(int32_t dt) { return dt == NVFP4_F32 || dt == NVFP4_BF16; }
 inline cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
 
+// Workspace layout: [0, 4) device error word, then kMaxAmaxCtas fp32
+// partial maxima per tensor from 256 on.  Nothing in it needs clearing.
 uint32_t* err_word(void* ws) { return static_cast<uint32_t*>(ws); }
-uint32_t* amax_slots(void* ws) {
-  return reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + kErrWordBytes);
+float* partials(void* ws) {
+  return reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kErrWordBytes);
 }
 
 // Shape / alignment rules of one quantizer input.
@@ -59,7 +61,8 @@ void fill_batch_common(QBatch& b, int32_t dtype, const nvfp4_qparams* qp, void* 
   b.block_axis = qp->block_axis;
   b.sf_layout = qp->sf_layout;
   b.gs_in = qp->global_scale_in;
-  b.amax_slots = ws ? amax_slots(ws) : nullptr;
+  b.partials = ws ? partials(ws) : nullptr;
+  b.err = ws ? err_word(ws) : nullptr;
 }
 
 nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
@@ -77,15 +80,10 @@ nvfp4_status quantize_common(const void* x, int32_t dtype, int64_t rows, int64_t
   if (!ws || ws_bytes < nvfp4_workspace_bytes(1)) return NVFP4_ERR_WORKSPACE;
   QBatch b;
   fill_batch_common(b, dtype, qp, ws);
+  b.two_d = two_d ? 1 : 0;
   b.n = 1;
   b.t[0] = QTensor{x, codes, scales, gs_out, rows, cols, ld};
-  if (!qp->global_scale_in) {
-    cudaError_t e = cudaMemsetAsync(amax_slots(ws), 0, sizeof(uint32_t), S(stream));
-    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
-    e = launch_amax(b, S(stream));
-    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
-  }
-  return cuda_status(two_d ? launch_quantize_2d(b, S(stream)) : launch_quantize_1d(b, S(stream)));
+  return cuda_status(launch_quantize(b, S(stream)));
 }
 
 }  // namespace
@@ -94,7 +92,7 @@ extern "C" {
 
 size_t nvfp4_workspace_bytes(int32_t n_tensors) {
   if (n_tensors < 0) n_tensors = 0;
-  return kErrWordBytes + ((size_t)n_tensors * 4 + 255) / 256 * 256;
+  return kErrWordBytes + (size_t)n_tensors * kMaxAmaxCtas * sizeof(float);
 }
 
 int64_t nvfp4_codes_bytes(int64_t rows, int64_t cols) { return rows * cols / 2; }
@@ -118,15 +116,11 @@ nvfp4_status nvfp4_global_scale(const void* x, int32_t dtype, int64_t rows, int6
   QBatch b;
   fill_batch_common(b, dtype, qp, ws);
   b.gs_in = nullptr;
+  b.amax_only = 1;
   b.n = 1;
   b.t[0] = QTensor{x, nullptr, nullptr, global_scale_out, rows, cols, ld};
-  cudaError_t e = cudaMemsetAsync(amax_slots(ws), 0, sizeof(uint32_t), S(stream));
-  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
-  if (rows > 0 && cols > 0) {
-    e = launch_amax(b, S(stream));
-    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
-  }
-  return cuda_status(launch_finalize_alpha(amax_slots(ws), global_scale_out, S(stream)));
+  // an empty tensor runs the same two kernels: amax 0, global scale 1
+  return cuda_status(launch_quantize(b, S(stream)));
 }
 
 nvfp4_status nvfp4_quantize_1d(const void* x, int32_t dtype, int64_t rows, int64_t cols,
@@ -163,21 +157,16 @@ nvfp4_status nvfp4_quantize_1d_batched(const nvfp4_tensor_desc* descs, int32_t n
   }
   if (!ws || ws_bytes < nvfp4_workspace_bytes(n)) return NVFP4_ERR_WORKSPACE;
   if (n == 0) return NVFP4_OK;
-  cudaError_t e = cudaMemsetAsync(amax_slots(ws), 0, sizeof(uint32_t) * (size_t)n, S(stream));
-  if (e != cudaSuccess) return NVFP4_ERR_CUDA;
   for (int32_t base = 0; base < n; base += kMaxBatch) {
     QBatch b;
     fill_batch_common(b, dtype, qp, ws);
-    b.amax_slots = amax_slots(ws) + base;
+    b.partials = partials(ws) + (size_t)base * kMaxAmaxCtas;
     b.n = (n - base) < kMaxBatch ? (n - base) : kMaxBatch;
     for (int32_t i = 0; i < b.n; ++i) {
       const nvfp4_tensor_desc& d = descs[base + i];
       b.t[i] = QTensor{d.x, d.codes, d.scales, d.global_scale, d.rows, d.cols, d.ld};
     }
-    e = launch_amax(b, S(stream));
-    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
-    e = launch_quantize_1d(b, S(stream));
-    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (launch_quantize(b, S(stream)) != cudaSuccess) return NVFP4_ERR_CUDA;
   }
   return NVFP4_OK;
 }

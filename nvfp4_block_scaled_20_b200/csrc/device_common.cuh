@@ -53,6 +53,21 @@ __device__ __forceinline__ void load16(const __nv_bfloat16* p, float v[16]) {
     v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
 }
+// 16 consecutive bf16 as 8 raw words (element 2i in the low half of word i).
+__device__ __forceinline__ void load16_raw(const __nv_bfloat16* p, uint32_t w[8]) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]),
+                 "=r"(w[6]), "=r"(w[7])
+               : "l"(p));
+}
+
+// max(|a|, |b|) per bf16 half (sign bits cleared; an exact selection).
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a & 0x7FFF7FFFu), "r"(b & 0x7FFF7FFFu));
+  return r;
+}
+
 __device__ __forceinline__ void load16(const float* p, float v[16]) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -163,9 +178,171 @@ __device__ __forceinline__ float tree16(const uint64_t e[8]) {
   return __fadd_rn(lo, hi);
 }
 
-// One candidate encoding of a 16-element row segment under scale s > 0:
-// codes (8 bytes, element 2j in the low nibble of byte j) and the row's
-// squared error.  s == 0 encodes all +0 with error sum(y^2).
+// Codes of correctly rounded quotients without dividing every element.
+//
+// q = RN(x * r), with r the hardware reciprocal of the divisor (at most one
+// ulp off), is within 2^-22 (relative) of the correctly rounded quotient Q.
+// The E2M1 and E4M3 conversions are monotone, so if the conversions of
+// q*(1 - 2^-20) and q*(1 + 2^-20) -- an interval that contains Q -- give the
+// same code, that is the code of Q.  Only when the two differ (Q within about
+// 2^-20 of a rounding boundary of the target format, ~0.1% of elements) is
+// the quotient computed with an IEEE division.
+constexpr float kUp = 1.0f + 0x1p-20f, kDn = 1.0f - 0x1p-20f;
+
+__device__ __forceinline__ float rcp_approx(float s) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+  return r;
+}
+
+// Range where the reciprocal bound above is established (no flush to zero).
+__device__ __forceinline__ bool rcp_ok(float s) { return s >= 0x1p-125f && s <= 0x1p+125f; }
+
+// Eight fp32 -> four bytes of E2M1 code pairs in one word (element 2j in the
+// low nibble of byte j), round to nearest even, saturating.
+__device__ __forceinline__ uint32_t cvt8_e2m1(const float a[8]) {
+  uint32_t r;
+  asm("{ .reg .b8 b0, b1, b2, b3;\n"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n"
+      "mov.b32 %0, {b0, b1, b2, b3}; }"
+      : "=r"(r)
+      : "f"(a[0]), "f"(a[1]), "f"(a[2]), "f"(a[3]), "f"(a[4]), "f"(a[5]), "f"(a[6]), "f"(a[7]));
+  return r;
+}
+
+// Word of four E2M1 code pairs -> eight exact fp32 values.
+__device__ __forceinline__ void dec8_e2m1(uint32_t w, float v[8]) {
+  uint32_t h[4];
+  asm("{ .reg .b8 b0, b1, b2, b3;\n"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n"
+      "cvt.rn.f16x2.e2m1x2 %3, b3; }"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(w));
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    v[2 * k] = __half2float(__ushort_as_half((unsigned short)(h[k] & 0xFFFFu)));
+    v[2 * k + 1] = __half2float(__ushort_as_half((unsigned short)(h[k] >> 16)));
+  }
+}
+
+// E2M1 codes of RN(y/s) for 8 elements (s > 0) as one word.
+__device__ __forceinline__ uint32_t codes8_exact(const float* y, float s) {
+  float q[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(y[i], s);
+  return cvt8_e2m1(q);
+}
+
+// Redo, with IEEE divisions, the code pairs of one 8-element word whose two
+// bracket conversions disagree (diff = ca ^ cb, nonzero bytes mark them).
+// Out of line: a call cannot be if-converted, so the rare exact path costs
+// nothing when it is not taken.
+static __device__ __noinline__ uint32_t fix_word_call(uint32_t ca, uint32_t diff, float y0, float y1,
+                                               float y2, float y3, float y4, float y5, float y6,
+                                               float y7, float s) {
+  const float y[8] = {y0, y1, y2, y3, y4, y5, y6, y7};
+  uint32_t w = ca;
+#pragma unroll 1
+  for (int k = 0; k < 4; ++k) {
+    if ((diff >> (8 * k)) & 0xFFu) {
+      const uint32_t b = f32x2_to_e2m1x2(__fdiv_rn(y[2 * k], s), __fdiv_rn(y[2 * k + 1], s));
+      w = (w & ~(0xFFu << (8 * k))) | (b << (8 * k));
+    }
+  }
+  return w;
+}
+
+// E2M1 codes of RN(y/s) for 16 elements (s > 0) as two words.  Pairs whose
+// bracket conversions disagree (about 1% of pairs on activations) are redone
+// exactly by fix_word_call.
+__device__ __forceinline__ void codes16(const float y[16], float s, uint32_t w[2]) {
+  if (rcp_ok(s)) {
+    const float r = rcp_approx(s);
+    const uint64_t rr = pack2(r, r), up = pack2(kUp, kUp), dn = pack2(kDn, kDn);
+    uint32_t diff[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float a[8], b[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint64_t q = mul2(pack2(y[8 * h + 2 * k], y[8 * h + 2 * k + 1]), rr);
+        unpack2(mul2(q, up), a[2 * k], a[2 * k + 1]);
+        unpack2(mul2(q, dn), b[2 * k], b[2 * k + 1]);
+      }
+      w[h] = cvt8_e2m1(a);
+      diff[h] = w[h] ^ cvt8_e2m1(b);
+    }
+    if (diff[0] | diff[1]) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        if (diff[h])
+          w[h] = fix_word_call(w[h], diff[h], y[8 * h], y[8 * h + 1], y[8 * h + 2], y[8 * h + 3],
+                               y[8 * h + 4], y[8 * h + 5], y[8 * h + 6], y[8 * h + 7], s);
+    }
+    return;
+  }
+  w[0] = codes8_exact(y, s);
+  w[1] = codes8_exact(y + 8, s);
+}
+
+// Two fp32 -> two E4M3 codes (a in bits 8-15, b in bits 0-7), RN, saturating.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float a, float b) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// Per-tensor constants for the candidate scale codes.
+struct ScaleCtx {
+  float alpha;
+  float c6, c4;  // ~ 1/(6 alpha), 1/(4 alpha)
+  bool fast;
+};
+
+__device__ __forceinline__ ScaleCtx make_scale_ctx(float alpha) {
+  ScaleCtx c;
+  c.alpha = alpha;
+  c.fast = rcp_ok(alpha);
+  const float ia = c.fast ? rcp_approx(alpha) : 0.0f;
+  c.c6 = __fmul_rn(ia, 1.0f / 6.0f);
+  c.c4 = __fmul_rn(ia, 0.25f);
+  return c;
+}
+
+// Exact E4M3 codes of the two candidate scales (out of line; see codes16).
+static __device__ __noinline__ uint2 scale_codes_exact_call(float bmax, float alpha) {
+  const float u = __fdiv_rn(bmax, alpha);
+  return make_uint2(f32_to_e4m3(__fdiv_rn(u, 6.0f)), f32_to_e4m3(__fmul_rn(u, 0.25f)));
+}
+
+// E4M3 codes of t6 = RN(RN(bmax / alpha) / 6) and t4 = RN(bmax / alpha) / 4.
+__device__ __forceinline__ void scale_codes(float bmax, const ScaleCtx& c, uint32_t& e6,
+                                            uint32_t& e4) {
+  bool exact = !c.fast;
+  if (!exact) {
+    const float t6 = __fmul_rn(bmax, c.c6), t4 = __fmul_rn(bmax, c.c4);
+    const uint32_t p6 = f32x2_to_e4m3x2(__fmul_rn(t6, kUp), __fmul_rn(t6, kDn));
+    const uint32_t p4 = f32x2_to_e4m3x2(__fmul_rn(t4, kUp), __fmul_rn(t4, kDn));
+    e6 = p6 & 0xFFu;
+    e4 = p4 & 0xFFu;
+    exact = ((p6 >> 8) != e6) || ((p4 >> 8) != e4);
+  }
+  if (exact) {  // out of line, as in codes16
+    const uint2 e = scale_codes_exact_call(bmax, c.alpha);
+    e6 = e.x;
+    e4 = e.y;
+  }
+}
+
+// One candidate encoding of a 16-element row segment under scale s:
+// codes (8 bytes) and the row's squared error sum (y - val(q) * s)^2.
+// s == 0 encodes all +0 with error sum(y^2).
 struct Cand {
   uint32_t lo, hi;  // packed codes
   float err;
@@ -177,51 +354,49 @@ __device__ __forceinline__ Cand encode16(const float y[16], float s) {
   if (s == 0.0f) {
     c.lo = c.hi = 0u;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) sq[k] = pack2(__fmul_rn(y[2 * k], y[2 * k]), __fmul_rn(y[2 * k + 1], y[2 * k + 1]));
+    for (int k = 0; k < 8; ++k)
+      sq[k] = pack2(__fmul_rn(y[2 * k], y[2 * k]), __fmul_rn(y[2 * k + 1], y[2 * k + 1]));
   } else {
-    uint32_t bytes[8];
+    uint32_t w[2];
+    codes16(y, s, w);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      float q0 = __fdiv_rn(y[2 * k], s);
-      float q1 = __fdiv_rn(y[2 * k + 1], s);
-      bytes[k] = f32x2_to_e2m1x2(q0, q1);
-      float v0, v1;
-      unpack2(e2m1x2_to_f32x2(bytes[k]), v0, v1);
-      // Scalar intrinsics: documented never to be merged into a fused
-      // multiply-add (the packed f32x2 forms are contracted by the
-      // assembler, which would change y - v*s in its last bit).
-      const float r0 = __fsub_rn(y[2 * k], __fmul_rn(v0, s));
-      const float r1 = __fsub_rn(y[2 * k + 1], __fmul_rn(v1, s));
-      sq[k] = pack2(__fmul_rn(r0, r0), __fmul_rn(r1, r1));
+    for (int h = 0; h < 2; ++h) {
+      float v[8];
+      dec8_e2m1(w[h], v);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        // Scalar intrinsics: documented never to be merged into a fused
+        // multiply-add (the packed f32x2 forms are contracted by the
+        // assembler, which would change y - v*s in its last bit).
+        const float r0 = __fsub_rn(y[8 * h + 2 * k], __fmul_rn(v[2 * k], s));
+        const float r1 = __fsub_rn(y[8 * h + 2 * k + 1], __fmul_rn(v[2 * k + 1], s));
+        sq[4 * h + k] = pack2(__fmul_rn(r0, r0), __fmul_rn(r1, r1));
+      }
     }
-    c.lo = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
-    c.hi = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
+    c.lo = w[0];
+    c.hi = w[1];
   }
   c.err = tree16(sq);
   return c;
 }
 
-// Scale of one candidate: t = (bmax / alpha) / M, e = E4M3(t), s = dec(e) * alpha.
-__device__ __forceinline__ float cand_scale(float u, float M, float alpha, uint32_t& e) {
-  float t = __fdiv_rn(u, M);
-  e = f32_to_e4m3(t);
+// Candidate scale s = dec(e) * alpha.
+__device__ __forceinline__ float cand_scale(uint32_t e, float alpha) {
   return __fmul_rn(e4m3_to_f32(e), alpha);
 }
 
 // Full 1D block encoding with the optional 4-vs-6 pick (ties keep 6).
-__device__ __forceinline__ void quantize_block16(const float y[16], float alpha, bool four_over_six,
-                                                 uint32_t& lo, uint32_t& hi, uint32_t& scale) {
-  const float u = __fdiv_rn(absmax16(y), alpha);
-  uint32_t e6;
-  const float s6 = cand_scale(u, 6.0f, alpha, e6);
-  Cand c6 = encode16(y, s6);
+__device__ __forceinline__ void quantize_block16(const float y[16], const ScaleCtx& ctx,
+                                                 bool four_over_six, uint32_t& lo, uint32_t& hi,
+                                                 uint32_t& scale) {
+  uint32_t e6, e4;
+  scale_codes(absmax16(y), ctx, e6, e4);
+  Cand c6 = encode16(y, cand_scale(e6, ctx.alpha));
   lo = c6.lo;
   hi = c6.hi;
   scale = e6;
   if (four_over_six) {
-    uint32_t e4;
-    const float s4 = cand_scale(u, 4.0f, alpha, e4);
-    Cand c4 = encode16(y, s4);
+    Cand c4 = encode16(y, cand_scale(e4, ctx.alpha));
     if (c4.err < c6.err) {
       lo = c4.lo;
       hi = c4.hi;

@@ -8,6 +8,9 @@
 namespace nvfp4 {
 
 constexpr int kMaxBatch = 64;  // tensors per batched launch (kernel parameter space)
+// Per-CTA partial maxima of the amax pass: at most this many CTAs per tensor,
+// one fp32 slot each in the workspace.
+constexpr int kMaxAmaxCtas = 320;
 
 struct QTensor {
   const void* x;
@@ -28,8 +31,11 @@ struct QBatch {
   uint32_t mask;
   int32_t block_axis;
   int32_t sf_layout;
-  const float* gs_in;   // device; nullptr => from amax slots
-  uint32_t* amax_slots; // device, one per tensor (float bits), zeroed by the caller
+  int32_t two_d;        // 1: 16x16 tiles (block_axis 0, no RHT)
+  int32_t amax_only;    // 1: only the amax pass; writes the global scale
+  const float* gs_in;   // device; nullptr => from the amax pass
+  float* partials;      // device, kMaxAmaxCtas slots per tensor (amax pass output)
+  uint32_t* err;        // device error word
 };
 
 struct DQTensor {
@@ -65,14 +71,14 @@ struct GemmArgs {
 int num_sms();
 
 // Each returns a cudaError_t from the launch.
-cudaError_t launch_amax(const QBatch& b, cudaStream_t s);
-cudaError_t launch_quantize_1d(const QBatch& b, cudaStream_t s);
-cudaError_t launch_quantize_2d(const QBatch& b, cudaStream_t s);
+// Quantization: an amax kernel writing per-CTA partial maxima, then the
+// encode kernel (programmatic dependent launch) that reduces them into the
+// global scale; only the encode kernel when gs_in is given, only the amax
+// kernel and a finalize kernel when amax_only is set.
+cudaError_t launch_quantize(const QBatch& b, cudaStream_t s);
 cudaError_t launch_dequantize(const DQBatch& b, cudaStream_t s);
 cudaError_t launch_rht16(const void* x, int bf16, int64_t rows, int64_t cols, int64_t ld,
                          int block_axis, uint32_t mask, float* out, cudaStream_t s);
-// Writes a_FP32 from the amax slot of tensor 0 to gs_out (amax-only call).
-cudaError_t launch_finalize_alpha(const uint32_t* amax_slot, float* gs_out, cudaStream_t s);
 // Returns 0 on success, a cudaError_t value otherwise; sets *unsupported for
 // shapes this build does not handle.
 int launch_gemm(const GemmArgs& a, cudaStream_t s, bool* unsupported);

@@ -5,9 +5,10 @@
 // every device byte and forbids side allocations, code that must not call
 // cudaMalloc because it would synchronize the device in the middle of a
 // latency-critical loop, or a C caller that only holds the raw pointers of its
-// tensors.  For them the per-tensor amax slots live in the fixed array below,
-// which is part of the library's device image: every GPU that loads the
-// library holds these kNoAllocMaxTensors * 4 bytes until the process exits.
+// tensors.  For them the per-tensor scratch of the amax pass (one partial
+// maximum per amax CTA) lives in the fixed array below, which is part of the
+// library's device image: every GPU that loads the library holds its
+// 256 + kNoAllocMaxTensors * kMaxAmaxCtas * 4 bytes (~80 KB) until exit.
 #include <cstring>
 #include <mutex>
 
@@ -16,11 +17,13 @@
 
 namespace {
 
-constexpr int kNoAllocMaxTensors = 256;
+constexpr int kNoAllocMaxTensors = 64;
 constexpr int kMaxDevices = 64;
 
-// One amax slot (fp32 bits) per tensor of a call.
-static __device__ __align__(256) uint32_t g_noalloc_amax[kNoAllocMaxTensors];
+// [0] device error word; from [64] on, kMaxAmaxCtas partial maxima (fp32
+// bits) per tensor of a call.  Every slot a call reads it has written in the
+// same call, so nothing needs clearing.
+static __device__ __align__(256) uint32_t g_noalloc_amax[64 + kNoAllocMaxTensors * nvfp4::kMaxAmaxCtas];
 
 std::mutex g_mu;
 uint32_t* g_addr[kMaxDevices] = {};
@@ -70,9 +73,6 @@ extern "C" nvfp4_status nvfp4_quantize_1d_batched_noalloc(const nvfp4_tensor_des
   nvfp4_status st = scratch_address(&slots);
   if (st != NVFP4_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the array keeps the previous call's maxima: clear the slots this call uses
-  if (cudaMemsetAsync(slots, 0, sizeof(uint32_t) * (size_t)n, s) != cudaSuccess)
-    return NVFP4_ERR_CUDA;
   for (int32_t base = 0; base < n; base += kMaxBatch) {
     QBatch b;
     memset(&b, 0, sizeof(b));
@@ -83,14 +83,14 @@ extern "C" nvfp4_status nvfp4_quantize_1d_batched_noalloc(const nvfp4_tensor_des
     b.block_axis = 0;
     b.sf_layout = qp->sf_layout;
     b.gs_in = nullptr;
-    b.amax_slots = slots + base;
+    b.err = slots;
+    b.partials = reinterpret_cast<float*>(slots + 64) + (size_t)base * kMaxAmaxCtas;
     b.n = 0;
     for (int32_t i = base; i < n && i < base + kMaxBatch; ++i) {
       const nvfp4_tensor_desc& d = descs[i];
       b.t[b.n++] = QTensor{d.x, d.codes, d.scales, d.global_scale, d.rows, d.cols, d.ld};
     }
-    if (launch_amax(b, s) != cudaSuccess) return NVFP4_ERR_CUDA;
-    if (launch_quantize_1d(b, s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (launch_quantize(b, s) != cudaSuccess) return NVFP4_ERR_CUDA;
   }
   return NVFP4_OK;
 }

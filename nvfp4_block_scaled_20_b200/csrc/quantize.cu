@@ -1,12 +1,20 @@
 // sm_100a NVFP4 quantizers, dequantizer and standalone RHT16.
 //
 // Current scaling needs the whole-tensor amax before the first element can be
-// encoded, so a quantization is two HBM passes: an amax pass (1) and an
-// encode pass (2).  Both passes are grid-stride, one 16-element block per
-// thread per step, 256-bit coalesced loads; the encode pass writes 8 bytes
-// of codes per block and one scale byte in the requested layout.  Batched
-// calls (KV cache) carry up to kMaxBatch tensors in the kernel parameters,
-// one tensor per blockIdx.y, so one launch covers a whole cache per pass.
+// encoded, so a quantization is two passes, two kernels on one stream:
+//   amax:   grid-stride over the tensor (256-bit coalesced loads, several in
+//           flight per thread), one partial maximum per CTA written to its own
+//           workspace slot -- no atomics, nothing to clear between calls;
+//   encode: launched as a programmatic dependent of the amax kernel, so its
+//           launch overlaps the amax pass; it waits for the amax grid,
+//           reduces the partials into the global scale and encodes one
+//           16-element block per thread step (both 4-vs-6 candidates, 8 bytes
+//           of codes and one scale byte in the requested layout).
+// A tensor that fits in L2 is read from HBM once: the encode pass finds it in
+// L2.  Batched calls (KV cache) carry up to kMaxBatch tensors in the kernel
+// parameters, one tensor per blockIdx.y.
+#include <type_traits>
+
 #include "device_common.cuh"
 #include "kernels.h"
 
@@ -28,38 +36,94 @@ __device__ __forceinline__ float block_reduce_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
   }
+  __syncthreads();  // red[] may be reused by the next call
   return v;
 }
 
-__device__ __forceinline__ float tensor_alpha(const QBatch& p, int t) {
-  return p.gs_in ? *p.gs_in : alpha_from_amax(__uint_as_float(p.amax_slots[t]));
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Global scale of tensor t from the amax kernel's partials (ga of them);
+// call after pdl_wait().  Every thread of the CTA gets the value.
+__device__ float reduce_partials(const float* part, int ga) {
+  float m = 0.0f;
+  for (int i = threadIdx.x; i < ga; i += kThreads) m = fmaxf(m, part[i]);
+  m = block_reduce_max(m);
+  __shared__ float s_m;
+  if (threadIdx.x == 0) s_m = m;
+  __syncthreads();
+  return s_m;
 }
 
 // ------------------------------------------------------------------------
-// Pass 1: amax.  Blocks along the contiguous dim (block_axis 0).
+// Amax pass.
+
+// bf16 without the transform: the max stays on packed raw words.
+__device__ float amax_rows_bf16_raw(const QTensor& q) {
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(q.x);
+  const uint32_t kbpr = (uint32_t)(q.cols >> 4);
+  const uint64_t nblk = (uint64_t)q.rows * kbpr;
+  const uint64_t stride = (uint64_t)gridDim.x * kThreads;
+  uint32_t m2 = 0u;
+  for (uint64_t u = (uint64_t)blockIdx.x * kThreads + threadIdx.x; u < nblk; u += 4 * stride) {
+    uint32_t w[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint64_t uj = u + j * stride;
+      if (uj < nblk) {
+        const uint32_t r = (uint32_t)uj / kbpr, kb = (uint32_t)uj - r * kbpr;
+        load16_raw(x + (int64_t)r * q.ld + (int64_t)kb * 16, w[j]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[j][i] = 0u;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m2 = absmax_bf16x2(m2, w[j][i]);
+  }
+  return fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u));
+}
+
 template <typename T, bool RHT>
-__global__ void __launch_bounds__(kThreads) amax_rows_kernel(const __grid_constant__ QBatch p) {
-  const QTensor& q = p.t[blockIdx.y];
+__device__ float amax_rows(const QTensor& q, uint32_t mask) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value && !RHT) return amax_rows_bf16_raw(q);
   const T* x = static_cast<const T*>(q.x);
   const uint32_t kbpr = (uint32_t)(q.cols >> 4);
   const uint64_t nblk = (uint64_t)q.rows * kbpr;
+  const uint64_t stride = (uint64_t)gridDim.x * kThreads;
   float m = 0.0f;
-  for (uint64_t u = (uint64_t)blockIdx.x * kThreads + threadIdx.x; u < nblk;
-       u += (uint64_t)gridDim.x * kThreads) {
-    const uint32_t r = (uint32_t)u / kbpr, kb = (uint32_t)u - r * kbpr;
-    float v[16];
-    load16(x + (int64_t)r * q.ld + (int64_t)kb * 16, v);
-    if (RHT) rht16(v, p.mask);
-    m = fmaxf(m, absmax16(v));
+  // two blocks per thread per trip, both loads issued before any use
+  for (uint64_t u = (uint64_t)blockIdx.x * kThreads + threadIdx.x; u < nblk; u += 2 * stride) {
+    float v[2][16];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint64_t uj = u + j * stride;
+      if (uj < nblk) {
+        const uint32_t r = (uint32_t)uj / kbpr, kb = (uint32_t)uj - r * kbpr;
+        load16(x + (int64_t)r * q.ld + (int64_t)kb * 16, v[j]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[j][i] = 0.0f;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      if (RHT) rht16(v[j], mask);
+      m = fmaxf(m, absmax16(v[j]));
+    }
   }
-  m = block_reduce_max(m);
-  if (threadIdx.x == 0) atomic_max_nonneg(&p.amax_slots[blockIdx.y], m);
+  return m;
 }
 
-// Pass 1 for blocks along rows (block_axis 1): unit = (column pair, 64 rows).
+// Per-thread amax over the row-axis units (column pair x 64 rows), with the
+// RHT applied along rows when enabled.  Reads element pairs only, so it needs
+// no more than the row-axis path's 16-byte row alignment.
 template <typename T, bool RHT>
-__global__ void __launch_bounds__(kThreads) amax_cols_kernel(const __grid_constant__ QBatch p) {
-  const QTensor& q = p.t[blockIdx.y];
+__device__ float amax_cols(const QTensor& q, uint32_t mask) {
   const T* x = static_cast<const T*>(q.x);
   const uint32_t ncp = (uint32_t)((q.cols + 1) >> 1);
   const uint32_t nrc = (uint32_t)((q.rows + 63) >> 6);
@@ -77,15 +141,13 @@ __global__ void __launch_bounds__(kThreads) amax_cols_kernel(const __grid_consta
 #pragma unroll
       for (int j = 0; j < 16; ++j) load2(x + (rg + j) * q.ld + c0, a[j], b[j]);
       if (RHT) {
-        rht16(a, p.mask);
-        rht16(b, p.mask);
+        rht16(a, mask);
+        rht16(b, mask);
       }
-      m = fmaxf(m, absmax16(a));
-      m = fmaxf(m, absmax16(b));
+      m = fmaxf(m, fmaxf(absmax16(a), absmax16(b)));
     }
   }
-  m = block_reduce_max(m);
-  if (threadIdx.x == 0) atomic_max_nonneg(&p.amax_slots[blockIdx.y], m);
+  return m;
 }
 
 // Zero the padding entries of a tcgen05-layout scale buffer.
@@ -107,18 +169,14 @@ __device__ void zero_sf_padding(uint8_t* sf, int64_t rows, int64_t kbpr) {
   }
 }
 
-// ------------------------------------------------------------------------
-// Pass 2: encode, blocks along the contiguous dim.
+// Encode pass, 16-blocks along the contiguous dim.
 template <typename T, bool RHT>
-__global__ void __launch_bounds__(kThreads) quant_rows_kernel(const __grid_constant__ QBatch p) {
-  const int t = blockIdx.y;
-  const QTensor& q = p.t[t];
+__device__ void encode_rows(const QTensor& q, float alpha, const QBatch& p) {
   const T* x = static_cast<const T*>(q.x);
-  const float alpha = tensor_alpha(p, t);
-  if (blockIdx.x == 0 && threadIdx.x == 0 && q.gs_out) *q.gs_out = alpha;
   const uint32_t kbpr = (uint32_t)(q.cols >> 4);
   const uint64_t nblk = (uint64_t)q.rows * kbpr;
   const bool fos = p.four_over_six != 0;
+  const ScaleCtx ctx = make_scale_ctx(alpha);
   for (uint64_t u = (uint64_t)blockIdx.x * kThreads + threadIdx.x; u < nblk;
        u += (uint64_t)gridDim.x * kThreads) {
     const uint32_t r = (uint32_t)u / kbpr, kb = (uint32_t)u - r * kbpr;
@@ -126,7 +184,7 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const __grid_const
     load16(x + (int64_t)r * q.ld + (int64_t)kb * 16, v);
     if (RHT) rht16(v, p.mask);
     uint32_t lo, hi, sc;
-    quantize_block16(v, alpha, fos, lo, hi, sc);
+    quantize_block16(v, ctx, fos, lo, hi, sc);
     *reinterpret_cast<uint2*>(q.codes + (int64_t)r * (q.cols >> 1) + (int64_t)kb * 8) =
         make_uint2(lo, hi);
     q.scales[sf_offset(r, kb, kbpr, p.sf_layout)] = (uint8_t)sc;
@@ -134,21 +192,18 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const __grid_const
   if (p.sf_layout == 1) zero_sf_padding(q.scales, q.rows, kbpr);
 }
 
-// Pass 2, blocks along rows; output transposed: codes [cols, rows/2],
-// scales for cols rows x rows/16 blocks.
+// Encode pass, blocks along rows; output transposed: codes [cols, rows/2],
+// scales for cols rows x rows/16 blocks.  Unit = column pair x 64 rows.
 template <typename T, bool RHT>
-__global__ void __launch_bounds__(kThreads) quant_cols_kernel(const __grid_constant__ QBatch p) {
-  const int t = blockIdx.y;
-  const QTensor& q = p.t[t];
+__device__ void encode_cols(const QTensor& q, float alpha, const QBatch& p) {
   const T* x = static_cast<const T*>(q.x);
-  const float alpha = tensor_alpha(p, t);
-  if (blockIdx.x == 0 && threadIdx.x == 0 && q.gs_out) *q.gs_out = alpha;
   const uint32_t ncp = (uint32_t)((q.cols + 1) >> 1);
   const uint32_t nrc = (uint32_t)((q.rows + 63) >> 6);
   const uint64_t nunits = (uint64_t)ncp * nrc;
   const int64_t out_row_bytes = q.rows >> 1;
   const int64_t kb_total = q.rows >> 4;
   const bool fos = p.four_over_six != 0;
+  const ScaleCtx ctx = make_scale_ctx(alpha);
   for (uint64_t u = (uint64_t)blockIdx.x * kThreads + threadIdx.x; u < nunits;
        u += (uint64_t)gridDim.x * kThreads) {
     const uint32_t rc = (uint32_t)u / ncp, cp = (uint32_t)u - rc * ncp;
@@ -165,10 +220,10 @@ __global__ void __launch_bounds__(kThreads) quant_cols_kernel(const __grid_const
         rht16(b, p.mask);
       }
       uint32_t lo, hi, sc;
-      quantize_block16(a, alpha, fos, lo, hi, sc);
+      quantize_block16(a, ctx, fos, lo, hi, sc);
       *reinterpret_cast<uint2*>(q.codes + c0 * out_row_bytes + (rg >> 1)) = make_uint2(lo, hi);
       q.scales[sf_offset(c0, rg >> 4, kb_total, p.sf_layout)] = (uint8_t)sc;
-      quantize_block16(b, alpha, fos, lo, hi, sc);
+      quantize_block16(b, ctx, fos, lo, hi, sc);
       *reinterpret_cast<uint2*>(q.codes + (c0 + 1) * out_row_bytes + (rg >> 1)) =
           make_uint2(lo, hi);
       q.scales[sf_offset(c0 + 1, rg >> 4, kb_total, p.sf_layout)] = (uint8_t)sc;
@@ -177,23 +232,20 @@ __global__ void __launch_bounds__(kThreads) quant_cols_kernel(const __grid_const
   if (p.sf_layout == 1) zero_sf_padding(q.scales, q.cols, kb_total);
 }
 
-// ------------------------------------------------------------------------
-// 2D 16x16 tiles.  A warp holds two adjacent tiles of one 16-row band: lane l
-// owns row (l & 15) of tile (l >> 4).  Tile max and tile error reduce across
-// the 16 lanes of a half-warp with xor shuffles 8, 4, 2, 1 -- the same
-// pairwise order as the per-row sum.
+// Encode pass, 16x16 tiles.  A warp holds two adjacent tiles of one 16-row
+// band: lane l owns row (l & 15) of tile (l >> 4).  Tile max and tile error
+// reduce across the 16 lanes of a half-warp with xor shuffles 8, 4, 2, 1 --
+// the same pairwise order as the per-row sum.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) quant_2d_kernel(const __grid_constant__ QBatch p) {
-  const QTensor& q = p.t[0];
+__device__ void encode_2d(const QTensor& q, float alpha, const QBatch& p) {
   const T* x = static_cast<const T*>(q.x);
-  const float alpha = tensor_alpha(p, 0);
-  if (blockIdx.x == 0 && threadIdx.x == 0 && q.gs_out) *q.gs_out = alpha;
   const uint32_t kbpr = (uint32_t)(q.cols >> 4);
   const uint32_t npair = (kbpr + 1) >> 1;
   const uint32_t nunits = (uint32_t)(q.rows >> 4) * npair;
   const int lane = threadIdx.x & 31;
   const uint32_t warps = kThreads / 32;
   const bool fos = p.four_over_six != 0;
+  const ScaleCtx ctx = make_scale_ctx(alpha);
   for (uint32_t u = blockIdx.x * warps + (threadIdx.x >> 5); u < nunits; u += gridDim.x * warps) {
     const uint32_t tr = u / npair, tp = u - tr * npair;
     const int64_t r = (int64_t)tr * 16 + (lane & 15);
@@ -209,18 +261,15 @@ __global__ void __launch_bounds__(kThreads) quant_2d_kernel(const __grid_constan
     float tmax = absmax16(v);
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xFFFFFFFFu, tmax, o));
-    const float uu = __fdiv_rn(tmax, alpha);
-    uint32_t e6;
-    const float s6 = cand_scale(uu, 6.0f, alpha, e6);
-    Cand c6 = encode16(v, s6);
+    uint32_t e6, e4;
+    scale_codes(tmax, ctx, e6, e4);
+    Cand c6 = encode16(v, cand_scale(e6, alpha));
     float err6 = c6.err;
 #pragma unroll
     for (int o = 8; o > 0; o >>= 1) err6 = __fadd_rn(err6, __shfl_xor_sync(0xFFFFFFFFu, err6, o));
     uint32_t lo = c6.lo, hi = c6.hi, sc = e6;
     if (fos) {
-      uint32_t e4;
-      const float s4 = cand_scale(uu, 4.0f, alpha, e4);
-      Cand c4 = encode16(v, s4);
+      Cand c4 = encode16(v, cand_scale(e4, alpha));
       float err4 = c4.err;
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) err4 = __fadd_rn(err4, __shfl_xor_sync(0xFFFFFFFFu, err4, o));
@@ -236,6 +285,60 @@ __global__ void __launch_bounds__(kThreads) quant_2d_kernel(const __grid_constan
     }
   }
   if (p.sf_layout == 1) zero_sf_padding(q.scales, q.rows, kbpr);
+}
+
+enum { kModeRows = 0, kModeCols = 1, kMode2D = 2 };
+
+// One CTA of the amax pass over tensor blockIdx.y: its partial maximum goes to
+// partials[t * kMaxAmaxCtas + blockIdx.x].
+template <typename T, int MODE, bool RHT>
+__global__ void __launch_bounds__(kThreads) amax_kernel(const __grid_constant__ QBatch p) {
+  const int t = blockIdx.y;
+  // the row-axis mode reads its input as element pairs in both passes: its
+  // rows need not satisfy the contiguous path's 32-byte alignment
+  float m = MODE == kModeCols ? amax_cols<T, RHT>(p.t[t], p.mask) : amax_rows<T, RHT>(p.t[t], p.mask);
+  m = block_reduce_max(m);
+  if (threadIdx.x == 0) p.partials[t * kMaxAmaxCtas + blockIdx.x] = m;
+  pdl_trigger();
+}
+
+// Global scale only: one CTA per tensor reduces the partials.
+__global__ void __launch_bounds__(kThreads) finalize_kernel(const __grid_constant__ QBatch p, int ga) {
+  pdl_wait();
+  const int t = blockIdx.x;
+  const float a = alpha_from_amax(reduce_partials(p.partials + t * kMaxAmaxCtas, ga));
+  if (threadIdx.x == 0 && p.t[t].gs_out) *p.t[t].gs_out = a;
+}
+
+// Encode pass over tensor blockIdx.y.  ga = number of amax partials (0 when
+// the global scale is given).
+template <typename T, int MODE, bool RHT>
+__global__ void __launch_bounds__(kThreads, 4) encode_kernel(const __grid_constant__ QBatch p, int ga) {
+  const int t = blockIdx.y;
+  float alpha;
+  if (p.gs_in) {
+    alpha = *p.gs_in;
+  } else {
+    pdl_wait();
+    alpha = alpha_from_amax(reduce_partials(p.partials + t * kMaxAmaxCtas, ga));
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0 && p.t[t].gs_out) *p.t[t].gs_out = alpha;
+  if (MODE == kModeRows) encode_rows<T, RHT>(p.t[t], alpha, p);
+  else if (MODE == kModeCols) encode_cols<T, RHT>(p.t[t], alpha, p);
+  else encode_2d<T>(p.t[t], alpha, p);
+}
+
+uint64_t max_units(const QBatch& b, int mode) {
+  uint64_t units = 0;
+  for (int i = 0; i < b.n; ++i) {
+    const QTensor& q = b.t[i];
+    // 16-blocks (rows), column pairs x 64 rows (cols), threads of 2-tile warps (2D)
+    uint64_t u = mode == kModeRows ? (uint64_t)q.rows * (uint64_t)(q.cols / 16)
+               : mode == kModeCols ? (uint64_t)((q.cols + 1) / 2) * (uint64_t)((q.rows + 63) / 64)
+                                   : (uint64_t)(q.rows / 16) * (uint64_t)((q.cols / 16 + 1) / 2) * 32;
+    units = u > units ? u : units;
+  }
+  return units;
 }
 
 // ------------------------------------------------------------------------
@@ -313,26 +416,11 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-__global__ void finalize_alpha_kernel(const uint32_t* slot, float* gs_out) {
-  *gs_out = alpha_from_amax(__uint_as_float(*slot));
-}
-
 int grid_for(uint64_t work_items, int n_tensors) {
   const uint64_t want = (work_items + kThreads - 1) / kThreads;
   const uint64_t cap = (uint64_t)num_sms() * 8 / (uint64_t)(n_tensors > 0 ? n_tensors : 1);
   uint64_t g = want < cap ? want : cap;
   return (int)(g < 1 ? 1 : g);
-}
-
-uint64_t max_units(const QBatch& b, bool cols_units) {
-  uint64_t m = 0;
-  for (int i = 0; i < b.n; ++i) {
-    const QTensor& q = b.t[i];
-    const uint64_t u = cols_units ? (uint64_t)((q.cols + 1) / 2) * (uint64_t)((q.rows + 63) / 64)
-                                  : (uint64_t)q.rows * (uint64_t)(q.cols / 16);
-    m = u > m ? u : m;
-  }
-  return m;
 }
 
 }  // namespace
@@ -348,47 +436,57 @@ int num_sms() {
   return n;
 }
 
-cudaError_t launch_amax(const QBatch& b, cudaStream_t s) {
-  const bool cols = b.block_axis == 1;
-  dim3 grid(grid_for(max_units(b, cols), b.n), b.n);
-#define NVFP4_AMAX(T, R)                                                            \
-  (cols ? amax_cols_kernel<T, R><<<grid, kThreads, 0, s>>>(b)                        \
-        : amax_rows_kernel<T, R><<<grid, kThreads, 0, s>>>(b))
-  if (b.bf16) {
-    if (b.rht) NVFP4_AMAX(__nv_bfloat16, true); else NVFP4_AMAX(__nv_bfloat16, false);
-  } else {
-    if (b.rht) NVFP4_AMAX(float, true); else NVFP4_AMAX(float, false);
-  }
-#undef NVFP4_AMAX
-  return cudaGetLastError();
+namespace {
+
+template <typename K, typename... Args>
+cudaError_t launch_ex(K kern, dim3 grid, cudaStream_t s, bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-cudaError_t launch_quantize_1d(const QBatch& b, cudaStream_t s) {
-  const bool cols = b.block_axis == 1;
-  dim3 grid(grid_for(max_units(b, cols), b.n), b.n);
-#define NVFP4_Q1(T, R)                                                              \
-  (cols ? quant_cols_kernel<T, R><<<grid, kThreads, 0, s>>>(b)                       \
-        : quant_rows_kernel<T, R><<<grid, kThreads, 0, s>>>(b))
-  if (b.bf16) {
-    if (b.rht) NVFP4_Q1(__nv_bfloat16, true); else NVFP4_Q1(__nv_bfloat16, false);
-  } else {
-    if (b.rht) NVFP4_Q1(float, true); else NVFP4_Q1(float, false);
+template <typename T, int MODE, bool RHT>
+cudaError_t launch_mode(const QBatch& b, cudaStream_t s) {
+  const uint64_t units = max_units(b, MODE);
+  const uint64_t per_cta = (uint64_t)kThreads;
+  int ga = 0;
+  if (!b.gs_in) {
+    // amax pass: at most two CTAs per SM (up to four loads in flight per thread)
+    uint64_t want = (units + 4 * per_cta - 1) / (4 * per_cta);
+    uint64_t cap = (uint64_t)num_sms() * 2;
+    if (cap > (uint64_t)kMaxAmaxCtas) cap = kMaxAmaxCtas;
+    ga = (int)(want < 1 ? 1 : (want < cap ? want : cap));
+    cudaError_t e = launch_ex(amax_kernel<T, MODE, RHT>, dim3(ga, b.n), s, false, b);
+    if (e != cudaSuccess) return e;
+    if (b.amax_only) return launch_ex(finalize_kernel, dim3(b.n), s, true, b, ga);
   }
-#undef NVFP4_Q1
-  return cudaGetLastError();
+  uint64_t cap = (uint64_t)num_sms() * 4 / (uint64_t)b.n;
+  if (cap < 1) cap = 1;
+  uint64_t want = (units + per_cta - 1) / per_cta;
+  const unsigned gx = (unsigned)(want < 1 ? 1 : (want < cap ? want : cap));
+  return launch_ex(encode_kernel<T, MODE, RHT>, dim3(gx, b.n), s, !b.gs_in, b, ga);
 }
 
-cudaError_t launch_quantize_2d(const QBatch& b, cudaStream_t s) {
-  const QTensor& q = b.t[0];
-  const uint64_t units = (uint64_t)(q.rows / 16) * (uint64_t)((q.cols / 16 + 1) / 2);
-  // one warp per unit: 8 units per CTA
-  uint64_t want = (units + 7) / 8, cap = (uint64_t)num_sms() * 8;
-  int grid = (int)(want < cap ? (want < 1 ? 1 : want) : cap);
-  if (b.bf16)
-    quant_2d_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(b);
-  else
-    quant_2d_kernel<float><<<grid, kThreads, 0, s>>>(b);
-  return cudaGetLastError();
+template <typename T>
+cudaError_t launch_typed(const QBatch& b, cudaStream_t s) {
+  if (b.two_d) return launch_mode<T, kMode2D, false>(b, s);
+  if (b.block_axis == 1)
+    return b.rht ? launch_mode<T, kModeCols, true>(b, s) : launch_mode<T, kModeCols, false>(b, s);
+  return b.rht ? launch_mode<T, kModeRows, true>(b, s) : launch_mode<T, kModeRows, false>(b, s);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const QBatch& b, cudaStream_t s) {
+  return b.bf16 ? launch_typed<__nv_bfloat16>(b, s) : launch_typed<float>(b, s);
 }
 
 cudaError_t launch_dequantize(const DQBatch& b, cudaStream_t s) {
@@ -418,9 +516,5 @@ cudaError_t launch_rht16(const void* x, int bf16, int64_t rows, int64_t cols, in
   return cudaGetLastError();
 }
 
-cudaError_t launch_finalize_alpha(const uint32_t* amax_slot, float* gs_out, cudaStream_t s) {
-  finalize_alpha_kernel<<<1, 1, 0, s>>>(amax_slot, gs_out);
-  return cudaGetLastError();
-}
 
 }  // namespace nvfp4

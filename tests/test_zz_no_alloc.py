@@ -68,6 +68,6 @@ def test_noalloc_matches_workspace_entry_point_twice():
 def test_noalloc_rejects_more_tensors_than_its_scratch():
     from nvfp4_block_scaled_20_b200 import build, capi
     build.build()
-    d = (capi.nvfp4_tensor_desc * 257)()
+    d = (capi.nvfp4_tensor_desc * 65)()
     qp = capi.nvfp4_qparams(1, 0, 0, 0, 0, 0, None)
-    assert capi.nvfp4_quantize_1d_batched_noalloc(d, 257, capi.NVFP4_BF16, qp, None) == 2
+    assert capi.nvfp4_quantize_1d_batched_noalloc(d, 65, capi.NVFP4_BF16, qp, None) == 2
