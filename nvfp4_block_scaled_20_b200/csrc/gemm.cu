@@ -3,17 +3,23 @@
 //   out[m, n] = epi(alpha_a * alpha_b * sum_k a_mk * sA[m, k/16] * b_nk * sB[n, k/16])
 //
 // A [M, K] and B [N, K] are packed E2M1 codes (K-major), sA / sB are UE4M3
-// scales in the tcgen05 block-scaled layout.  One CTA computes a 128 x BN
-// tile of the output:
+// scales in the tcgen05 block-scaled layout.  Persistent kernel: one CTA per
+// SM walks 128 x 256 output tiles in a grouped (L2-friendly) order.
 //   warp 0      TMA producer: codes with cp.async.bulk.tensor (128B swizzle),
-//               scale atoms with cp.async.bulk, into a STAGES-deep ring;
-//   warp 1      allocates tensor memory and issues, from one thread, the
-//               tcgen05.cp of the stage's scale atoms into tensor memory and
-//               the tcgen05.mma kind::mxf4nvf4 (block16 scales, K = 64 each);
-//               tcgen05.commit releases the smem stage;
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (one row per
-//               thread), x alpha_a*alpha_b, optional GELU(tanh), bf16 / fp32
-//               stores.
+//               scale atoms with cp.async.bulk, into a 4-deep ring that runs
+//               ahead across tile boundaries;
+//   warp 1      allocates tensor memory; one thread issues, per MMA k-block,
+//               the tcgen05.cp of its scale atoms into a 12-column slot and
+//               the tcgen05.mma kind::mxf4nvf4 (block16 scales, K = 64);
+//               tcgen05.commit releases ring stages and signals accumulators;
+//   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulator (two warps per
+//               32-lane quadrant, half of the columns each), x alpha_a*alpha_b,
+//               optional GELU(tanh), bf16 / fp32 stores.
+// Tensor memory holds two 256-column accumulators and one MMA k-block's scale
+// factors (12 columns): 524 of the 512 columns, so the second accumulator
+// starts at column 240 and the two share 16 columns.  The epilogue drains the
+// shared columns first and releases them, so the next tile's MMAs wait only
+// for that, not for the whole drain.
 // Every wait is bounded (wall clock through %globaltimer); on a timeout the
 // CTA records NVFP4_ERR_TIMEOUT in the device error word, drains what it
 // issued and frees its tensor memory before returning.
@@ -26,27 +32,29 @@ namespace nvfp4 {
 
 namespace {
 
-constexpr int BM = 128;           // rows per CTA tile (one TMEM lane per row)
+constexpr int BM = 128;           // rows per tile (one TMEM lane per row)
+constexpr int BN = 256;           // columns per tile
 constexpr int BK = 256;           // K elements per stage = 128 bytes of codes per row
 constexpr int BK_BYTES = BK / 2;  // one 128-byte swizzle row
 constexpr int MMA_K = 64;         // K per tcgen05.mma (kind::mxf4nvf4)
-constexpr int kNumThreads = 192;
+constexpr int kStages = 4;
+constexpr int kEpiWarps = 8;
+constexpr int kNumThreads = (2 + kEpiWarps) * 32;
+constexpr int kABytes = BM * BK_BYTES;          // 16 KB
+constexpr int kBBytes = BN * BK_BYTES;          // 32 KB
+constexpr int kSfaBytes = 4 * 512;              // 4 atoms (128 rows x 16 blocks)
+constexpr int kSfbBytes = (BN / 128) * 4 * 512;
+constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+// tensor memory columns
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAcc1Col = 240;   // accumulator 0 at column 0, 1 at 240
+constexpr uint32_t kOvlCols = 16;    // columns [240, 256) belong to both
+constexpr uint32_t kSfaCol = 496;    // 4 columns: one MMA k-block of A scales
+constexpr uint32_t kSfbCol = 500;    // 8 columns: one MMA k-block of B scales
+constexpr int kGroupM = 8;           // tile raster: 8 M-tiles per group
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s when draining after an abort
-
-template <int BN>
-struct Cfg {
-  static constexpr int kStages = BN == 256 ? 4 : 6;
-  static constexpr int kABytes = BM * BK_BYTES;               // 16 KB
-  static constexpr int kBBytes = BN * BK_BYTES;               // 16 / 32 KB
-  static constexpr int kSfaBytes = 4 * 512;                   // 4 atoms (128 rows x 16 blocks)
-  static constexpr int kSfbBytes = (BN / 128) * 4 * 512;
-  static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-  static constexpr int kTmemCols = BN == 256 ? 512 : 256;     // accumulator + scale factors
-  static constexpr int kSfaCol = BN;                          // 4 MMAs x 4 columns
-  static constexpr int kSfbCol = BN + 16;                     // 4 MMAs x (BN/32) columns
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
-};
 
 // --------------------------------------------------------------- PTX wrappers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -63,6 +71,9 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -184,35 +195,79 @@ struct Params {
   uint32_t* err;
 };
 
-template <int BN>
+// Tile t of the grouped raster -> (tile row, tile column).
+__device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mt, int& nt) {
+  const int per_group = kGroupM * num_n;
+  const int g = t / per_group;
+  const int first_m = g * kGroupM;
+  const int gm = min(kGroupM, num_m - first_m);
+  const int r = t - g * per_group;
+  mt = first_m + r % gm;
+  nt = r / gm;
+}
+
+__device__ __forceinline__ void store16(const Params& p, int row, int col, const uint32_t r[16],
+                                        float scale) {
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    v[i] = __fmul_rn(__uint_as_float(r[i]), scale);
+    if (p.epilogue == 1) v[i] = gelu_tanh(v[i]);
+  }
+  if (p.out_bf16) {
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    uint4* d4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + (int64_t)row * p.ldo + col);
+    d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  } else {
+    float4* d4 = reinterpret_cast<float4*>(static_cast<float*>(p.out) + (int64_t)row * p.ldo + col);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  }
+}
+
 __global__ void __launch_bounds__(kNumThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ Params p) {
-  using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = smem;
-  uint8_t* sB = sA + C::kStages * C::kABytes;
-  uint8_t* sSFA = sB + C::kStages * C::kBBytes;
-  uint8_t* sSFB = sSFA + C::kStages * C::kSfaBytes;
-  uint64_t* bars = (uint64_t*)(sSFB + C::kStages * C::kSfbBytes);
-  uint64_t* full = bars;                    // [kStages]
-  uint64_t* empty = bars + C::kStages;      // [kStages]
-  uint64_t* accum = bars + 2 * C::kStages;  // [1]
-  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * C::kStages + 1);
+  uint8_t* sB = sA + kStages * kABytes;
+  uint8_t* sSFA = sB + kStages * kBBytes;
+  uint8_t* sSFB = sSFA + kStages * kSfaBytes;
+  uint64_t* bars = (uint64_t*)(sSFB + kStages * kSfbBytes);
+  uint64_t* full = bars;                        // [kStages]   TMA -> MMA
+  uint64_t* empty = bars + kStages;             // [kStages]   MMA -> TMA
+  uint64_t* acc_full = bars + 2 * kStages;      // [2]         MMA -> epilogue
+  uint64_t* acc_empty = bars + 2 * kStages + 2; // [2]         epilogue -> MMA
+  uint64_t* ovl_free = bars + 2 * kStages + 4;  // [1]         shared columns drained
+  uint64_t* mma_done = bars + 2 * kStages + 5;  // [1]         all MMAs of this CTA done
+  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * kStages + 6);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  const int num_m = (p.M + BM - 1) / BM, num_n = (p.N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
   const int num_kt = (p.K + BK - 1) / BK;
-  const int kgroups = p.K / 64;  // 4-block scale groups per row band
+  const int kgroups = p.K / 64;  // 4-block scale groups per 128-row band
+  const int nbands_total = (p.N + 127) / 128;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1);
     }
-    mbar_init(smem_u32(accum), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&acc_full[b]), 1);
+      mbar_init(smem_u32(&acc_empty[b]), kEpiWarps);
+    }
+    mbar_init(smem_u32(ovl_free), kEpiWarps / 2);
+    mbar_init(smem_u32(mma_done), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -220,7 +275,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
-                 "r"(C::kTmemCols)
+                 "r"(kTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -228,130 +283,153 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // operands may be written by the preceding kernel (programmatic launch)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int issued = 0;
+      uint32_t it = 0;
       bool ok = true;
-      for (int kt = 0; kt < num_kt && ok; ++kt) {
-        const int s = kt % C::kStages;
-        const uint32_t round = (uint32_t)(kt / C::kStages);
-        if (!mbar_wait(smem_u32(&empty[s]), (round & 1u) ^ 1u, abort_flag, kWaitLimitNs)) {
-          ok = false;
-          break;
-        }
-        const int atoms = min(4, kgroups - kt * 4);
-        uint32_t bytes = C::kABytes + C::kBBytes + atoms * 512;
-        const int nbands_total = (p.N + 127) / 128;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        int mt, nt;
+        tile_coords(t, num_m, num_n, mt, nt);
+        const int m0 = mt * BM, n0 = nt * BN;
         int bands = 0;
         for (int b = 0; b < BN / 128; ++b)
           if (n0 / 128 + b < nbands_total) ++bands;
-        bytes += bands * atoms * 512;
-        const uint32_t fb = smem_u32(&full[s]);
-        mbar_expect_tx(fb, bytes);
-        tma_load_2d(smem_u32(sA + s * C::kABytes), &tmA, kt * BK_BYTES, m0, fb);
-        tma_load_2d(smem_u32(sB + s * C::kBBytes), &tmB, kt * BK_BYTES, n0, fb);
-        bulk_load(smem_u32(sSFA + s * C::kSfaBytes),
-                  p.a_sf + ((int64_t)(m0 / 128) * kgroups + kt * 4) * 512, atoms * 512, fb);
-        for (int b = 0; b < bands; ++b)
-          bulk_load(smem_u32(sSFB + s * C::kSfbBytes + b * 2048),
-                    p.b_sf + ((int64_t)(n0 / 128 + b) * kgroups + kt * 4) * 512, atoms * 512, fb);
-        issued = kt + 1;
+        for (int kt = 0; kt < num_kt; ++kt, ++it) {
+          const int s = it % kStages;
+          const uint32_t round = it / kStages;
+          if (!mbar_wait(smem_u32(&empty[s]), (round & 1u) ^ 1u, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          const int atoms = min(4, kgroups - kt * 4);
+          const uint32_t bytes = kABytes + kBBytes + atoms * 512 * (1 + bands);
+          const uint32_t fb = smem_u32(&full[s]);
+          mbar_expect_tx(fb, bytes);
+          tma_load_2d(smem_u32(sA + s * kABytes), &tmA, kt * BK_BYTES, m0, fb);
+          tma_load_2d(smem_u32(sB + s * kBBytes), &tmB, kt * BK_BYTES, n0, fb);
+          bulk_load(smem_u32(sSFA + s * kSfaBytes),
+                    p.a_sf + ((int64_t)(m0 / 128) * kgroups + kt * 4) * 512, atoms * 512, fb);
+          for (int b = 0; b < bands; ++b)
+            bulk_load(smem_u32(sSFB + s * kSfbBytes + b * 2048),
+                      p.b_sf + ((int64_t)(n0 / 128 + b) * kgroups + kt * 4) * 512, atoms * 512, fb);
+        }
       }
       if (!ok) {
         *abort_flag = 1;
         atomicOr(p.err, kDevErrTimeout);
       }
-      // Drain: every stage this thread issued must have landed before the
-      // CTA can retire (bounded).
-      for (int kt = (issued > C::kStages ? issued - C::kStages : 0); kt < issued; ++kt) {
-        const int s = kt % C::kStages;
-        mbar_wait(smem_u32(&full[s]), (uint32_t)(kt / C::kStages) & 1u, nullptr, kDrainLimitNs);
-      }
+      // every stage issued must have landed before the CTA retires (bounded)
+      for (uint32_t j = (it > (uint32_t)kStages ? it - kStages : 0u); j < it; ++j)
+        mbar_wait(smem_u32(&full[j % kStages]), (j / kStages) & 1u, nullptr, kDrainLimitNs);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = instr_desc(BM, BN);
-      const uint32_t t_acc = tmem;
-      const uint32_t t_sfa = tmem + C::kSfaCol;
-      const uint32_t t_sfb = tmem + C::kSfbCol;
+      const uint32_t t_sfa = tmem + kSfaCol, t_sfb = tmem + kSfbCol;
+      uint32_t it = 0, tile_i = 0;
       bool ok = true;
-      for (int kt = 0; kt < num_kt; ++kt) {
-        const int s = kt % C::kStages;
-        if (!mbar_wait(smem_u32(&full[s]), (uint32_t)(kt / C::kStages) & 1u, abort_flag,
-                       kWaitLimitNs)) {
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++tile_i) {
+        const uint32_t b = tile_i & 1u, use = tile_i >> 1;
+        // accumulator b drained by the epilogue of tile_i - 2, and the shared
+        // columns by the epilogue of tile_i - 1
+        if (use > 0 && !mbar_wait(smem_u32(&acc_empty[b]), (use - 1) & 1u, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        if (tile_i > 0 && !mbar_wait(smem_u32(ovl_free), (tile_i - 1) & 1u, abort_flag, kWaitLimitNs)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int nmma = min(4, (p.K - kt * BK) / MMA_K);
-        const uint32_t a_base = smem_u32(sA + s * C::kABytes);
-        const uint32_t b_base = smem_u32(sB + s * C::kBBytes);
-        const uint32_t sfa_base = smem_u32(sSFA + s * C::kSfaBytes);
-        const uint32_t sfb_base = smem_u32(sSFB + s * C::kSfbBytes);
-        for (int k = 0; k < nmma; ++k) {
-          tc_cp_sf(t_sfa + 4 * k, sf_desc(sfa_base + 512 * k));
-#pragma unroll
-          for (int b = 0; b < BN / 128; ++b)
-            tc_cp_sf(t_sfb + (BN / 32) * k + 4 * b, sf_desc(sfb_base + 2048 * b + 512 * k));
+        const uint32_t t_acc = tmem + (b ? kAcc1Col : 0u);
+        for (int kt = 0; kt < num_kt; ++kt, ++it) {
+          const int s = it % kStages;
+          if (!mbar_wait(smem_u32(&full[s]), (it / kStages) & 1u, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nmma = min(4, (p.K - kt * BK) / MMA_K);
+          const uint32_t a_base = smem_u32(sA + s * kABytes);
+          const uint32_t b_base = smem_u32(sB + s * kBBytes);
+          const uint32_t sfa_base = smem_u32(sSFA + s * kSfaBytes);
+          const uint32_t sfb_base = smem_u32(sSFB + s * kSfbBytes);
+          for (int k = 0; k < nmma; ++k) {
+            // tcgen05 operations from one thread execute in issue order: the
+            // copy into the scale slot waits for the previous MMA's reads
+            tc_cp_sf(t_sfa, sf_desc(sfa_base + 512 * k));
+            tc_cp_sf(t_sfb, sf_desc(sfb_base + 512 * k));
+            tc_cp_sf(t_sfb + 4, sf_desc(sfb_base + 2048 + 512 * k));
+            tc_mma(t_acc, operand_desc(a_base + 32 * k), operand_desc(b_base + 32 * k), idesc, t_sfa,
+                   t_sfb, (kt > 0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit(smem_u32(&empty[s]));
         }
-        for (int k = 0; k < nmma; ++k) {
-          tc_mma(t_acc, operand_desc(a_base + 32 * k), operand_desc(b_base + 32 * k), idesc,
-                 t_sfa + 4 * k, t_sfb + (BN / 32) * k, (kt > 0 || k > 0) ? 1u : 0u);
-        }
-        tc_commit(smem_u32(&empty[s]));
+        // signals once this tile's MMAs (and everything before) completed
+        tc_commit(smem_u32(&acc_full[b]));
       }
       if (!ok) {
         *abort_flag = 1;
         atomicOr(p.err, kDevErrTimeout);
       }
-      // Always signal the accumulator barrier: it completes once every
-      // tcgen05 operation issued above has finished.
-      tc_commit(smem_u32(accum));
+      // no MMA may still run when the CTA frees its tensor memory (bounded)
+      tc_commit(smem_u32(mma_done));
+      mbar_wait(smem_u32(mma_done), 0, nullptr, kWaitLimitNs);
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
-    const bool ok = mbar_wait(smem_u32(accum), 0, nullptr, kWaitLimitNs);
-    tc_fence_after();
-    if (ok && !*abort_flag) {
-      const float scale = __fmul_rn(*p.a_alpha, *p.b_alpha);
-      const int row = m0 + quad * 32 + lane;
-      const bool row_ok = row < p.M;
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, r);
-        const int col = n0 + c0;
-        if (!row_ok || col >= p.N) continue;
-        float v[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          v[i] = __fmul_rn(__uint_as_float(r[i]), scale);
-          if (p.epilogue == 1) v[i] = gelu_tanh(v[i]);
-        }
-        if (p.out_bf16) {
-          uint32_t w[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-            w[i] = *reinterpret_cast<uint32_t*>(&h);
-          }
-          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + (int64_t)row * p.ldo + col;
-          uint4* d4 = reinterpret_cast<uint4*>(dst);
-          d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        } else {
-          float* dst = static_cast<float*>(p.out) + (int64_t)row * p.ldo + col;
-          float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-        }
+    const int e = warp - 2;        // 0..7
+    const int quad = warp & 3;     // TMEM lanes 32*quad .. 32*quad+31
+    const int half = e >> 2;       // columns [128*half, 128*half + 128)
+    const float scale = __fmul_rn(*p.a_alpha, *p.b_alpha);
+    uint32_t tile_i = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tile_i) {
+      const uint32_t b = tile_i & 1u, use = tile_i >> 1;
+      int mt, nt;
+      tile_coords(t, num_m, num_n, mt, nt);
+      const int m0 = mt * BM, n0 = nt * BN;
+      if (!mbar_wait(smem_u32(&acc_full[b]), use & 1u, abort_flag, kWaitLimitNs)) {
+        atomicOr(p.err, kDevErrTimeout);
+        *abort_flag = 1;
+        break;
       }
-    } else if (!ok) {
-      atomicOr(p.err, kDevErrTimeout);
+      tc_fence_after();
+      const uint32_t t_acc = tmem + (b ? kAcc1Col : 0u) + ((uint32_t)(quad * 32) << 16);
+      const int row = m0 + quad * 32 + lane;
+      const bool quad_live = m0 + quad * 32 < p.M;  // warp-uniform
+      // the 16 columns shared with the other accumulator: tile columns
+      // 240..255 of accumulator 0, 0..15 of accumulator 1
+      const int ovl_half = b ? 0 : 1;
+      const int ovl_c0 = b ? 0 : 256 - (int)kOvlCols;
+      if (half == ovl_half) {
+#pragma unroll 1
+        for (int c = ovl_c0; c < ovl_c0 + (int)kOvlCols; c += 16) {
+          if (!quad_live || n0 + c >= p.N) continue;
+          uint32_t r[16];
+          tmem_ld16(t_acc + (uint32_t)c, r);
+          if (row < p.M) store16(p, row, n0 + c, r, scale);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(ovl_free));
+      }
+#pragma unroll 1
+      for (int j = 0; j < 8; ++j) {
+        const int c = half * 128 + j * 16;
+        if (half == ovl_half && c >= ovl_c0 && c < ovl_c0 + (int)kOvlCols) continue;
+        if (!quad_live || n0 + c >= p.N) continue;
+        uint32_t r[16];
+        tmem_ld16(t_acc + (uint32_t)c, r);
+        if (row < p.M) store16(p, row, n0 + c, r, scale);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
     }
   }
 
@@ -360,10 +438,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    // the accumulator barrier (bounded) guarantees no tcgen05 op is in flight
-    mbar_wait(smem_u32(accum), 0, nullptr, kDrainLimitNs);
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(C::kTmemCols)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                  : "memory");
   }
 }
@@ -402,9 +477,7 @@ bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_
   return r == CUDA_SUCCESS;
 }
 
-template <int BN>
-int launch_bn(const GemmArgs& a, cudaStream_t s) {
-  using C = Cfg<BN>;
+int launch_persistent(const GemmArgs& a, cudaStream_t s) {
   CUtensorMap tmA, tmB;
   if (!make_codes_map(&tmA, a.a_codes, a.M, a.K, BM)) return (int)cudaErrorInvalidValue;
   if (!make_codes_map(&tmB, a.b_codes, a.N, a.K, BN)) return (int)cudaErrorInvalidValue;
@@ -423,14 +496,24 @@ int launch_bn(const GemmArgs& a, cudaStream_t s) {
   p.err = a.err;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
     if (e != cudaSuccess) return (int)e;
     attr_set = true;
   }
-  dim3 grid((unsigned)((a.N + BN - 1) / BN), (unsigned)((a.M + BM - 1) / BM));
-  gemm_kernel<BN><<<grid, kNumThreads, C::kSmemBytes, s>>>(tmA, tmB, p);
-  return (int)cudaGetLastError();
+  const int64_t tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
+  const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kNumThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return (int)cudaLaunchKernelEx(&cfg, gemm_kernel, tmA, tmB, p);
 }
 
 }  // namespace
@@ -441,8 +524,7 @@ int launch_gemm(const GemmArgs& a, cudaStream_t s, bool* unsupported) {
     *unsupported = true;
     return 0;
   }
-  if (a.N <= 128) return launch_bn<128>(a, s);
-  return launch_bn<256>(a, s);
+  return launch_persistent(a, s);
 }
 
 }  // namespace nvfp4
