@@ -30,6 +30,8 @@ M, N, K = 2640, 9216, 3072
 WORKLOAD = "DiT QKV projection W4A4: X bf16 [2640x3072] (1% Student-t(3)x8 channels), " \
            "W bf16 [9216x3072] N(0,0.02); 1D act + 2D weight NVFP4, 4-vs-6 on; Y bf16 [2640x9216]"
 FLUSH_BYTES = 256 << 20
+# our kernels per step: amax + encode for X, amax + encode for W, the GEMM
+LAUNCHES_PER_STEP = 5
 # CPU-oracle sample: the first rows of the same workload
 CPU_MS, CPU_NS = 64, 128
 
@@ -213,6 +215,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--rows", default="auto", choices=["auto", "on", "off"],
+                    help="also time every hot-path row at its full workload size "
+                         "(auto: on a single GPU only)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args)
@@ -351,6 +356,12 @@ def main():
                 "L2, so its second read is served from L2.  Each line is timed after an L2 flush.",
     }
 
+    rows = None
+    if args.rows == "on" or (args.rows == "auto" and world == 1):
+        del graphs
+        rows = measure_rows(nv, synth, torch, dev, stream, timed, pk, reps)
+        graphs = None
+
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(nv, torch, dev, stream, x, w, qa, qb, ws_a, ws_b, ws_g, args, world)
@@ -377,9 +388,11 @@ def main():
                          "peak_source": "%s bf16 burst %.1f TFLOP/s x 4 (nominal dense FP4:BF16 "
                                         "ratio)" % (pk["source"], pk["bf16_tflops"])},
             "breakdown": breakdown,
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clk,
         }
+        if rows:
+            line["rows"] = rows
         if e2e:
             line["e2e"] = e2e
         if cpu:
@@ -390,6 +403,144 @@ def main():
         del graphs
         dist.destroy_process_group()
     return 0
+
+
+def measure_rows(nv, synth, torch, dev, stream, timed, pk, reps):
+    """Every hot-path row at its full workload size, same protocol as the step
+    (graph replay between CUDA events, L2 flushed before each replay):
+
+    a1 global amax, a3 1D quantize and a5 GEMMs on the DiT FFN pair (X
+    [8192, 3072], W_up [14336, 3072], W_dn [3072, 14336], H [8192, 14336]);
+    a4 2D quantize on both FFN weights; a2 RHT16 + transposing quantize and
+    the fp32 GEMM of the weight-gradient path (dY [32768, 3072], X [32768,
+    14336]); a6 batched quantize and a7 batched dequant of the 60-tensor KV
+    cache (30 layers x {K, V} x [24 * 32760, 128]).  Bytes are the
+    algorithmic ones: an input read by both passes counts twice."""
+    hbm = pk["hbm_gbs"]
+    fp4 = 4.0 * pk["bf16_tflops"]
+    T = nv.NVFP4_SF_TCGEN05
+    qout = 0.5 + 1.0 / 16
+
+    def graph(fn):
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                fn()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        return g
+
+    def bw(fn, nbytes, note=None):
+        ms = timed(graph(fn), reps)
+        v = nbytes / (ms * 1e-3) / 1e9
+        r = {"ms": round(ms, 5), "GB/s": round(v, 1), "frac_hbm": round(v / hbm, 3),
+             "bytes": int(nbytes)}
+        if note:
+            r["note"] = note
+        return r
+
+    def tc(fn, flops):
+        ms = timed(graph(fn), reps)
+        v = flops / (ms * 1e-3) / 1e12
+        return {"ms": round(ms, 5), "TFLOP/s": round(v, 1), "frac_fp4_peak": round(v / fp4, 3),
+                "flops": flops}
+
+    def q(rows, cols, layout=T):
+        return nv.QTensor(*nv._alloc_q(rows, cols, layout, dev), rows, cols, layout)
+
+    out = {}
+    ws = nv.workspace(1, dev)
+    # ---------------- FFN pair
+    x, wu, wd = synth.ffn_pair(dev)
+    Mf, D = x.shape
+    Hd = wu.shape[0]
+    qx, qu, qd, qh = q(Mf, D), q(Hd, D), q(D, Hd), q(Mf, Hd)
+    h = torch.empty((Mf, Hd), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((Mf, D), dtype=torch.bfloat16, device=dev)
+    nv.quantize_1d(x, out=qx, ws=ws, stream=stream)
+    nv.quantize_2d(wu, out=qu, ws=ws, stream=stream)
+    nv.quantize_2d(wd, out=qd, ws=ws, stream=stream)
+    nv.gemm(qx, qu, out=h, epilogue=nv.NVFP4_EPI_GELU_TANH, ws=ws, stream=stream)
+    ne_h = Mf * Hd
+    out["a1_global_amax"] = {
+        "H_8192x14336": bw(lambda: nv.global_scale(h, out=qh.alpha, ws=ws, stream=stream),
+                           2 * ne_h)}
+    out["a3_quantize_1d"] = {
+        "H_8192x14336": bw(lambda: nv.quantize_1d(h, out=qh, ws=ws, stream=stream),
+                           (4 + qout) * ne_h),
+        "H_8192x14336_encode_only": bw(
+            lambda: nv.quantize_1d(h, out=qh, ws=ws, alpha_in=qh.alpha, stream=stream),
+            (2 + qout) * ne_h),
+        "X_8192x3072": bw(lambda: nv.quantize_1d(x, out=qx, ws=ws, stream=stream),
+                          (4 + qout) * Mf * D, "50 MB input: its second read hits L2"),
+    }
+    out["a4_quantize_2d"] = {
+        "W_up_14336x3072": bw(lambda: nv.quantize_2d(wu, out=qu, ws=ws, stream=stream),
+                              (4 + qout) * Hd * D, "88 MB input: its second read hits L2"),
+        "W_dn_3072x14336": bw(lambda: nv.quantize_2d(wd, out=qd, ws=ws, stream=stream),
+                              (4 + qout) * Hd * D, "88 MB input: its second read hits L2"),
+    }
+    nv.quantize_1d(h, out=qh, ws=ws, stream=stream)
+    g_up = tc(lambda: nv.gemm(qx, qu, out=h, epilogue=nv.NVFP4_EPI_GELU_TANH, ws=ws,
+                              stream=stream), 2.0 * Mf * Hd * D)
+    g_dn = tc(lambda: nv.gemm(qh, qd, out=y, ws=ws, stream=stream), 2.0 * Mf * D * Hd)
+
+    def ffn_step():
+        nv.quantize_1d(x, out=qx, ws=ws, stream=stream)
+        nv.gemm(qx, qu, out=h, epilogue=nv.NVFP4_EPI_GELU_TANH, ws=ws, stream=stream)
+        nv.quantize_1d(h, out=qh, ws=ws, stream=stream)
+        nv.gemm(qh, qd, out=y, ws=ws, stream=stream)
+
+    ffn = tc(ffn_step, 4.0 * Mf * Hd * D)
+    ffn["note"] = "quantize X, up GEMM + GELU, quantize H, down GEMM (weights pre-quantized)"
+    del x, wu, wd, qx, qu, qd, qh, h, y
+
+    # ---------------- weight gradient
+    dy, xw, mask = synth.wgrad(dev)
+    Tk, Do = dy.shape
+    Di = xw.shape[1]
+    qdy, qxw = q(Do, Tk), q(Di, Tk)
+    dw = torch.empty((Do, Di), dtype=torch.float32, device=dev)
+    out["a2_rht16_transposed_quantize"] = {
+        "X_32768x14336": bw(lambda: nv.quantize_1d(xw, rht=True, mask=mask, block_axis=1,
+                                                   out=qxw, ws=ws, stream=stream),
+                            (4 + qout) * Tk * Di),
+        "dY_32768x3072": bw(lambda: nv.quantize_1d(dy, rht=True, mask=mask, block_axis=1,
+                                                   out=qdy, ws=ws, stream=stream),
+                            (4 + qout) * Tk * Do),
+    }
+    g_wg = tc(lambda: nv.gemm(qdy, qxw, out=dw, ws=ws, stream=stream), 2.0 * Do * Di * Tk)
+
+    def wgrad_step():
+        nv.quantize_1d(dy, rht=True, mask=mask, block_axis=1, out=qdy, ws=ws, stream=stream)
+        nv.quantize_1d(xw, rht=True, mask=mask, block_axis=1, out=qxw, ws=ws, stream=stream)
+        nv.gemm(qdy, qxw, out=dw, ws=ws, stream=stream)
+
+    wg = tc(wgrad_step, 2.0 * Do * Di * Tk)
+    wg["note"] = "RHT16 + transposing quantize of dY and X, fp32 GEMM"
+    out["a5_gemm"] = {"ffn_up_gelu_8192x14336x3072": g_up, "ffn_down_8192x3072x14336": g_dn,
+                      "wgrad_3072x14336x32768_fp32": g_wg}
+    out["steps"] = {"ffn_pair": ffn, "wgrad": wg}
+    del dy, xw, qdy, qxw, dw
+
+    # ---------------- KV cache
+    kv = [synth.kv_tensor(3, l, wh, device=dev) for l in range(30) for wh in range(2)]
+    R, C = kv[0].shape
+    kq = [q(R, C, nv.NVFP4_SF_ROWMAJOR) for _ in kv]
+    kout = [torch.empty((R, C), dtype=torch.bfloat16, device=dev) for _ in kv]
+    ws_kv = nv.workspace(len(kv), dev)
+    ne_kv = len(kv) * R * C
+    out["a6_kv_quantize_batched"] = bw(
+        lambda: nv.quantize_1d_batched(kv, outs=kq, ws=ws_kv, stream=stream),
+        (4 + qout) * ne_kv, "60 tensors, one amax launch + one encode launch")
+    out["a7_kv_dequant_batched"] = bw(
+        lambda: nv.dequantize(kq, outs=kout, stream=stream), (qout + 2) * ne_kv,
+        "60 tensors, one launch")
+    del kv, kq, kout
+    assert nv.device_error(ws, stream) == 0 and nv.device_error(ws_kv, stream) == 0
+    torch.cuda.empty_cache()
+    return out
 
 
 def measure_e2e(nv, torch, dev, stream, x, w, qa, qb, ws_a, ws_b, ws_g, args, world):
