@@ -206,6 +206,82 @@ def run_reference(args, world, rank):
     return 0
 
 
+# ------------------------------------------------------------------ ncu cases
+PROFILE_CASES = {
+    "qkv_step": "DiT QKV step: quantize X [2640, 3072], quantize W [9216, 3072], GEMM",
+    "h_quantize": "1D quantize of an FFN-hidden-sized bf16 [8192, 14336]: amax + encode, "
+                  "then encode alone (global scale given)",
+    "w_quantize_2d": "2D quantize of W_up [14336, 3072]",
+    "wgrad_x_quantize": "RHT16 + transposing quantize of X [8192, 14336] (a quarter of the "
+                        "weight-gradient tokens)",
+    "kv_quantize": "batched quantize + batched dequant of 4 KV tensors [24 * 32760, 128]",
+    "ffn_gemm": "FFN up GEMM + GELU 8192x14336x3072 and down GEMM 8192x3072x14336",
+    "wgrad_gemm": "weight-gradient GEMM 3072x14336x8192, fp32 out (a quarter of the tokens)",
+}
+
+
+def run_profile_case(name, reps=3):
+    """The case's kernels launched `reps` times on inputs generated once (a few
+    GB on the device at most)."""
+    import torch
+    import nvfp4_block_scaled_20_b200 as nv
+    from nvfp4_block_scaled_20_b200 import build, synth
+    build.build()
+    dev = torch.device("cuda", 0)
+    ws = nv.workspace(8, dev)
+
+    if name == "qkv_step":
+        x, w = synth.qkv_linear(dev)
+
+        def run():
+            nv.gemm(nv.quantize_1d(x, ws=ws), nv.quantize_2d(w, ws=ws), ws=ws)
+    elif name == "h_quantize":
+        h = synth.activation(2, 9, 8192, 14336, device=dev)
+        qh = nv.quantize_1d(h, ws=ws)
+
+        def run():
+            nv.quantize_1d(h, out=qh, ws=ws)
+            nv.quantize_1d(h, alpha_in=qh.alpha, out=qh, ws=ws)
+    elif name == "w_quantize_2d":
+        w = synth.weight(2, 2, 14336, 3072, device=dev)
+
+        def run():
+            nv.quantize_2d(w, ws=ws)
+    elif name == "wgrad_x_quantize":
+        x = synth.activation(4, 2, 8192, 14336, device=dev)
+
+        def run():
+            nv.quantize_1d(x, rht=True, mask=synth.rht_sign_mask(0), block_axis=1, ws=ws)
+    elif name == "kv_quantize":
+        kv = [synth.kv_tensor(3, l, wh, device=dev) for l in range(2) for wh in range(2)]
+
+        def run():
+            nv.dequantize(nv.quantize_1d_batched(kv, ws=ws))
+    elif name == "ffn_gemm":
+        x, wu, wd = synth.ffn_pair(dev)
+        qx, qu, qd = nv.quantize_1d(x, ws=ws), nv.quantize_2d(wu, ws=ws), nv.quantize_2d(wd, ws=ws)
+        h = torch.empty((x.shape[0], wu.shape[0]), dtype=torch.bfloat16, device=dev)
+        qh = nv.quantize_1d(h.zero_(), ws=ws)
+
+        def run():
+            nv.gemm(qx, qu, out=h, epilogue=nv.NVFP4_EPI_GELU_TANH, ws=ws)
+            nv.gemm(nv.quantize_1d(h, out=qh, ws=ws), qd, ws=ws)
+    else:  # wgrad_gemm
+        dy, xw, mask = synth.wgrad(dev, t=8192)
+        qdy = nv.quantize_1d(dy, rht=True, mask=mask, block_axis=1, ws=ws)
+        qxw = nv.quantize_1d(xw, rht=True, mask=mask, block_axis=1, ws=ws)
+
+        def run():
+            nv.gemm(qdy, qxw, out_dtype=torch.float32, ws=ws)
+
+    for _ in range(reps):
+        run()
+    torch.cuda.synchronize()
+    assert nv.device_error(ws) == 0
+    print("profile case %s: %s, %d reps" % (name, PROFILE_CASES[name], reps))
+    return 0
+
+
 # ------------------------------------------------------------------ GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -218,11 +294,16 @@ def main():
     ap.add_argument("--rows", default="auto", choices=["auto", "on", "off"],
                     help="also time every hot-path row at its full workload size "
                          "(auto: on a single GPU only)")
+    ap.add_argument("--profile", default=None, choices=sorted(PROFILE_CASES),
+                    help="run one small case a few times (untimed, no JSON line): the "
+                         "program the ncu captures under profiles/ are taken on")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup(args)
     if args.impl == "reference":
         return run_reference(args, world, rank)
+    if args.profile:
+        return run_profile_case(args.profile)
 
     import torch
     import nvfp4_block_scaled_20_b200 as nv
@@ -238,6 +319,8 @@ def main():
     if rank:
         x = synth.activation(1 + 1000 * rank, 1, M, K, device=dev)
         w = synth.weight(1 + 1000 * rank, 2, N, K, device=dev)
+    # the generator runs on torch's current stream, the path on `stream`
+    torch.cuda.synchronize(dev)
     qa = nv.QTensor(*nv._alloc_q(M, K, nv.NVFP4_SF_TCGEN05, dev), M, K, nv.NVFP4_SF_TCGEN05)
     qb = nv.QTensor(*nv._alloc_q(N, K, nv.NVFP4_SF_TCGEN05, dev), N, K, nv.NVFP4_SF_TCGEN05)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
@@ -453,6 +536,7 @@ def measure_rows(nv, synth, torch, dev, stream, timed, pk, reps):
     ws = nv.workspace(1, dev)
     # ---------------- FFN pair
     x, wu, wd = synth.ffn_pair(dev)
+    torch.cuda.synchronize(dev)  # generated on torch's current stream
     Mf, D = x.shape
     Hd = wu.shape[0]
     qx, qu, qd, qh = q(Mf, D), q(Hd, D), q(D, Hd), q(Mf, Hd)
@@ -498,6 +582,7 @@ def measure_rows(nv, synth, torch, dev, stream, timed, pk, reps):
 
     # ---------------- weight gradient
     dy, xw, mask = synth.wgrad(dev)
+    torch.cuda.synchronize(dev)
     Tk, Do = dy.shape
     Di = xw.shape[1]
     qdy, qxw = q(Do, Tk), q(Di, Tk)
@@ -526,6 +611,7 @@ def measure_rows(nv, synth, torch, dev, stream, timed, pk, reps):
 
     # ---------------- KV cache
     kv = [synth.kv_tensor(3, l, wh, device=dev) for l in range(30) for wh in range(2)]
+    torch.cuda.synchronize(dev)
     R, C = kv[0].shape
     kq = [q(R, C, nv.NVFP4_SF_ROWMAJOR) for _ in kv]
     kout = [torch.empty((R, C), dtype=torch.bfloat16, device=dev) for _ in kv]

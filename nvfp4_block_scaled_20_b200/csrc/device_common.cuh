@@ -38,6 +38,18 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
+// Packed subtract and fused multiply-add: only in approx_err16 below, whose
+// result is used with an error bound (contraction there is harmless).
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
 
 // ----------------------------------------------------------------- loads
 // 16 consecutive elements -> fp32.  bf16: one 256-bit load; fp32: two.
@@ -403,6 +415,151 @@ __device__ __forceinline__ void quantize_block16(const float y[16], const ScaleC
       scale = e4;
     }
   }
+}
+
+// ----------------------------------------------------------------- fast pick
+// The 4-vs-6 pick without the exact error sums in the common case.
+//
+// For a candidate with scale s > 0 (a normal E4M3 code, so that every
+// quotient Q = y/s is at most 6.4 and every residual |Q - v| at most 1):
+//  * the exact error E (fp32 products, differences, squares and the tree,
+//    as the encoding defines it) is within 304 * 2^-24 * s^2 of
+//    s^2 * sum (Q - v)^2 -- each of the 16 terms is off by at most
+//    15 * 2^-24 * s^2 and the four tree levels add 4 * 2^-24 of the sum;
+//  * approx_err16 (quotients through the hardware reciprocal, within 2^-18
+//    of Q; fused multiply-adds) is within 2^-12 of sum (Q - v)^2 -- each
+//    square is off by at most 2^-16, a boundary element that rounds the
+//    other way included, since both neighbours are then equally far.
+// So |E - s^2 * approx| < 2^-11.8 * s^2, and with the margin B = 2^-10 * s^2
+// the pick is certain when the two intervals [A - B, A + B] do not overlap.
+// Otherwise (and for zero or subnormal scale codes, or scales outside the
+// reciprocal's range) the block takes the exact path.
+constexpr float kPickMargin = 0x1p-10f;
+
+// The E2M1 values of a packed pair of quotients, as fp32x2 (exact): one
+// conversion to the code pair, one back to half precision, two widenings.
+__device__ __forceinline__ uint64_t e2m1_round_pair(uint64_t q) {
+  float lo, hi;
+  unpack2(q, lo, hi);
+  uint32_t h2;
+  asm("{ .reg .b8 c;\n"
+      "cvt.rn.satfinite.e2m1x2.f32 c, %1, %2;\n"
+      "cvt.rn.f16x2.e2m1x2 %0, c; }"
+      : "=r"(h2)
+      : "f"(hi), "f"(lo));
+  return pack2(__half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu))),
+               __half2float(__ushort_as_half((unsigned short)(h2 >> 16))));
+}
+
+// sum_i (q_i - v_i)^2 over 16 elements, q = y * r, v = the E2M1 value of q.
+__device__ __forceinline__ float approx_err16(const float y[16], float r) {
+  const uint64_t rr = pack2(r, r);
+  uint64_t acc[2] = {0ull, 0ull};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint64_t q = mul2(pack2(y[2 * k], y[2 * k + 1]), rr);
+    const uint64_t d = sub2(q, e2m1_round_pair(q));
+    acc[k & 1] = fma2(d, d, acc[k & 1]);
+  }
+  float a0, a1, b0, b1;
+  unpack2(acc[0], a0, a1);
+  unpack2(acc[1], b0, b1);
+  return (a0 + a1) + (b0 + b1);
+}
+
+// 0: keep the 6-candidate, 1: take the 4-candidate, 2: too close to call.
+__device__ __forceinline__ int certified_pick(float a6, float s6, float a4, float s4,
+                                              float margin) {
+  const float q6 = s6 * s6, q4 = s4 * s4;
+  const float A6 = a6 * q6, A4 = a4 * q4;
+  const float B = margin * (q6 + q4);
+  if (A4 + B < A6) return 1;
+  if (A4 > A6 + B) return 0;
+  return 2;
+}
+
+// Whether the fast pick applies to this pair of candidate scale codes.
+__device__ __forceinline__ bool fast_pick_ok(uint32_t e6, float s6, float s4) {
+  return e6 >= 8u && rcp_ok(s6) && rcp_ok(s4);  // e4 >= e6
+}
+
+// E2M1 codes of RN(y/s) for 16 elements from r = rcp_approx(s) (s in the
+// reciprocal's range), bracketed as in codes16: q*(1 +- 2^-20) becomes
+// y * (r*(1 +- 2^-20)), which still lies on the same side of the correctly
+// rounded quotient (the reciprocal is off by at most 2^-22, each product
+// rounds by 2^-24).  Returns false when a pair is ambiguous (the codes are
+// then to be redone exactly).
+__device__ __forceinline__ bool codes16_try(const float y[16], float r, uint32_t w[2]) {
+  const float ru = r * kUp, rd = r * kDn;
+  const uint64_t up = pack2(ru, ru), dn = pack2(rd, rd);
+  uint32_t diff = 0u;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float a[8], b[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint64_t yy = pack2(y[8 * h + 2 * k], y[8 * h + 2 * k + 1]);
+      unpack2(mul2(yy, up), a[2 * k], a[2 * k + 1]);
+      unpack2(mul2(yy, dn), b[2 * k], b[2 * k + 1]);
+    }
+    w[h] = cvt8_e2m1(a);
+    diff |= w[h] ^ cvt8_e2m1(b);
+  }
+  return diff == 0u;
+}
+
+// Scale codes by the bracket only; false when either is ambiguous.
+__device__ __forceinline__ bool scale_codes_try(float bmax, const ScaleCtx& c, uint32_t& e6,
+                                                uint32_t& e4) {
+  if (!c.fast) return false;
+  const float t6 = __fmul_rn(bmax, c.c6), t4 = __fmul_rn(bmax, c.c4);
+  const uint32_t p6 = f32x2_to_e4m3x2(__fmul_rn(t6, kUp), __fmul_rn(t6, kDn));
+  const uint32_t p4 = f32x2_to_e4m3x2(__fmul_rn(t4, kUp), __fmul_rn(t4, kDn));
+  e6 = p6 & 0xFFu;
+  e4 = p4 & 0xFFu;
+  return (p6 >> 8) == e6 && (p4 >> 8) == e4;
+}
+
+// Outcome of the fast block encoder.
+enum : uint32_t {
+  kBlockDone = 0,   // codes and scale final
+  kBlockCodes = 1,  // scale final; codes to be redone exactly with it
+  kBlockExact = 2,  // the whole block to be redone by quantize_block16
+};
+
+// One 16-element block through the fast path: bracketed scale codes, the
+// certified 4-vs-6 pick, bracketed codes of the winner.  Every result it
+// reports as final equals quantize_block16's; the rest it hands back.
+__device__ __forceinline__ uint32_t quantize_block16_try(const float y[16], const ScaleCtx& ctx,
+                                                         bool four_over_six, uint32_t& lo,
+                                                         uint32_t& hi, uint32_t& scale) {
+  uint32_t e6, e4;
+  if (!scale_codes_try(absmax16(y), ctx, e6, e4)) return kBlockExact;
+  const float s6 = cand_scale(e6, ctx.alpha);
+  uint32_t ew = e6;
+  float sw = s6;
+  if (four_over_six && e4 != e6) {  // equal codes: identical candidates, 6 wins the tie
+    const float s4 = cand_scale(e4, ctx.alpha);
+    if (!fast_pick_ok(e6, s6, s4)) return kBlockExact;
+    const int pick = certified_pick(approx_err16(y, rcp_approx(s6)), s6,
+                                    approx_err16(y, rcp_approx(s4)), s4, kPickMargin);
+    if (pick == 2) return kBlockExact;
+    if (pick == 1) {
+      ew = e4;
+      sw = s4;
+    }
+  }
+  scale = ew;
+  if (sw == 0.0f) {
+    lo = hi = 0u;
+    return kBlockDone;
+  }
+  if (!rcp_ok(sw)) return kBlockCodes;
+  uint32_t w[2];
+  const bool ok = codes16_try(y, rcp_approx(sw), w);
+  lo = w[0];
+  hi = w[1];
+  return ok ? kBlockDone : kBlockCodes;
 }
 
 // Byte offset of scale (r, kb) in the chosen layout.

@@ -45,6 +45,22 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// n / d for 32-bit n by a multiply-high (d fixed per tensor; d >= 1): with
+// l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1, n / d equals
+// (mulhi(n, m) + n) >> l for every 32-bit n.
+struct FastDiv {
+  uint32_t m, l;
+};
+__device__ __forceinline__ FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.l = d > 1u ? 32u - __clz(d - 1u) : 0u;
+  f.m = (uint32_t)(((((uint64_t)1 << f.l) - d) << 32) / d + 1u);
+  return f;
+}
+__device__ __forceinline__ uint32_t fastdiv(uint32_t n, FastDiv f) {
+  return (uint32_t)(((uint64_t)__umulhi(n, f.m) + n) >> f.l);
+}
+
 // Global scale of tensor t from the amax kernel's partials (ga of them);
 // call after pdl_wait().  Every thread of the CTA gets the value.
 __device__ float reduce_partials(const float* part, int ga) {
@@ -60,17 +76,20 @@ __device__ float reduce_partials(const float* part, int ga) {
 // ------------------------------------------------------------------------
 // Amax pass.
 
-// bf16 without the transform: the max stays on packed raw words.
+// bf16 without the transform: the max stays on packed raw words; kAmaxDepth
+// 32-byte loads in flight per thread (enough bytes in flight per SM to cover
+// the HBM latency at two CTAs per SM).
+constexpr int kAmaxDepth = 8;
 __device__ float amax_rows_bf16_raw(const QTensor& q) {
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(q.x);
   const uint32_t kbpr = (uint32_t)(q.cols >> 4);
   const uint64_t nblk = (uint64_t)q.rows * kbpr;
   const uint64_t stride = (uint64_t)gridDim.x * kThreads;
   uint32_t m2 = 0u;
-  for (uint64_t u = (uint64_t)blockIdx.x * kThreads + threadIdx.x; u < nblk; u += 4 * stride) {
-    uint32_t w[4][8];
+  for (uint64_t u = (uint64_t)blockIdx.x * kThreads + threadIdx.x; u < nblk; u += kAmaxDepth * stride) {
+    uint32_t w[kAmaxDepth][8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < kAmaxDepth; ++j) {
       const uint64_t uj = u + j * stride;
       if (uj < nblk) {
         const uint32_t r = (uint32_t)uj / kbpr, kb = (uint32_t)uj - r * kbpr;
@@ -81,7 +100,7 @@ __device__ float amax_rows_bf16_raw(const QTensor& q) {
       }
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < kAmaxDepth; ++j)
 #pragma unroll
       for (int i = 0; i < 8; ++i) m2 = absmax_bf16x2(m2, w[j][i]);
   }
@@ -119,27 +138,74 @@ __device__ float amax_rows(const QTensor& q, uint32_t mask) {
   return m;
 }
 
-// Per-thread amax over the row-axis units (column pair x 64 rows), with the
-// RHT applied along rows when enabled.  Reads element pairs only, so it needs
-// no more than the row-axis path's 16-byte row alignment.
+// 16 rows x one column pair (element pairs: the row-axis mode needs no more
+// than 4-byte row alignment), as loaded; widened to two fp32 columns.
+template <typename T> struct RawPair;
+template <> struct RawPair<__nv_bfloat16> {
+  uint32_t w[16];
+  __device__ __forceinline__ void load(const __nv_bfloat16* p, int64_t ld) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      asm volatile("ld.global.nc.b32 %0, [%1];" : "=r"(w[j]) : "l"(p + j * ld));
+  }
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) w[j] = 0u;
+  }
+  __device__ __forceinline__ void widen(float a[16], float b[16]) const {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      a[j] = __uint_as_float(w[j] << 16);
+      b[j] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  }
+};
+template <> struct RawPair<float> {
+  float2 f[16];
+  __device__ __forceinline__ void load(const float* p, int64_t ld) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) f[j] = __ldg(reinterpret_cast<const float2*>(p + j * ld));
+  }
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) f[j] = make_float2(0.0f, 0.0f);
+  }
+  __device__ __forceinline__ void widen(float a[16], float b[16]) const {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      a[j] = f[j].x;
+      b[j] = f[j].y;
+    }
+  }
+};
+
+// Per-thread amax over the row-axis units (column pair x 16 rows; rows % 16
+// == 0 and cols even for this mode), with the RHT applied along rows when
+// enabled; two units' loads in flight per thread.
 template <typename T, bool RHT>
 __device__ float amax_cols(const QTensor& q, uint32_t mask) {
   const T* x = static_cast<const T*>(q.x);
-  const uint32_t ncp = (uint32_t)((q.cols + 1) >> 1);
-  const uint32_t nrc = (uint32_t)((q.rows + 63) >> 6);
-  const uint64_t nunits = (uint64_t)ncp * nrc;
+  const uint32_t ncp = (uint32_t)(q.cols >> 1);
+  const uint32_t nunits = ncp * (uint32_t)(q.rows >> 4);
+  const FastDiv div = make_fastdiv(ncp);
+  const uint32_t stride = gridDim.x * kThreads;
   float m = 0.0f;
-  for (uint64_t u = (uint64_t)blockIdx.x * kThreads + threadIdx.x; u < nunits;
-       u += (uint64_t)gridDim.x * kThreads) {
-    const uint32_t rc = (uint32_t)u / ncp, cp = (uint32_t)u - rc * ncp;
-    const int64_t c0 = 2 * (int64_t)cp;
-#pragma unroll 1
-    for (int g = 0; g < 4; ++g) {
-      const int64_t rg = 64 * (int64_t)rc + 16 * g;
-      if (rg >= q.rows) break;
-      float a[16], b[16];
+  for (uint32_t u = blockIdx.x * kThreads + threadIdx.x; u < nunits; u += 2 * stride) {
+    RawPair<T> raw[2];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) load2(x + (rg + j) * q.ld + c0, a[j], b[j]);
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t uj = u + j * stride;
+      if (uj < nunits) {
+        const uint32_t rg = fastdiv(uj, div), cp = uj - rg * ncp;
+        raw[j].load(x + (int64_t)rg * 16 * q.ld + 2 * (int64_t)cp, q.ld);
+      } else {
+        raw[j].zero();
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float a[16], b[16];
+      raw[j].widen(a, b);
       if (RHT) {
         rht16(a, mask);
         rht16(b, mask);
@@ -169,85 +235,222 @@ __device__ void zero_sf_padding(uint8_t* sf, int64_t rows, int64_t kbpr) {
   }
 }
 
-// Encode pass, 16-blocks along the contiguous dim.
+// Raw 16-element block as loaded: bf16 keeps its 8 packed words, fp32 its 16
+// values; widened to fp32 when used.
+template <typename T> struct RawBlock;
+template <> struct RawBlock<__nv_bfloat16> {
+  uint32_t w[8];
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { load16_raw(p, w); }
+  __device__ __forceinline__ void widen(float v[16]) const {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+};
+template <> struct RawBlock<float> {
+  float f[16];
+  __device__ __forceinline__ void load(const float* p) { load16(p, f); }
+  __device__ __forceinline__ void widen(float v[16]) const {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = f[i];
+  }
+};
+
+// Blocks the fast encoder hands back are queued per warp (block index and
+// the final scale code, or kRedoAll) and redone exactly by the whole warp
+// when the queue fills and at the end, so a rare block does not stall the
+// other 31 lanes at every step.
+constexpr int kQueueCap = 128;            // entries per warp
+constexpr uint32_t kRedoAll = 0xFFFFFFFFu;  // redo the pick as well
+
+struct WarpQueue {
+  uint2* item;  // shared memory, kQueueCap entries
+  uint32_t n;   // same value on every lane
+  __device__ __forceinline__ void push(bool need, uint32_t idx, uint32_t code) {
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
+    if (need) item[n + __popc(m & ((1u << (threadIdx.x & 31)) - 1u))] = make_uint2(idx, code);
+    n += __popc(m);
+  }
+  template <typename F>
+  __device__ __forceinline__ void drain(F&& redo) {
+    __syncwarp();
+    for (uint32_t i = threadIdx.x & 31; i < n; i += 32) redo(item[i]);
+    __syncwarp();
+    n = 0;
+  }
+};
+
+__device__ __forceinline__ void store_codes(uint8_t* dst, uint32_t lo, uint32_t hi) {
+  *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+}
+
+// The exact encoding of one block for a queued entry: the whole block
+// (kRedoAll) or its codes under the given final scale code.
+__device__ __forceinline__ void redo_block(const float v[16], uint32_t code, const ScaleCtx& ctx,
+                                           bool fos, uint8_t* codes_dst, uint8_t* scale_dst) {
+  uint32_t lo, hi, sc;
+  if (code == kRedoAll) {
+    quantize_block16(v, ctx, fos, lo, hi, sc);
+    *scale_dst = (uint8_t)sc;
+  } else {
+    uint32_t w[2];
+    codes16(v, cand_scale(code, ctx.alpha), w);
+    lo = w[0];
+    hi = w[1];
+  }
+  store_codes(codes_dst, lo, hi);
+}
+
+// Encode pass, 16-blocks along the contiguous dim.  CTA-uniform grid-stride
+// over blocks, the next block's load issued before the current one is
+// encoded.
 template <typename T, bool RHT>
-__device__ void encode_rows(const QTensor& q, float alpha, const QBatch& p) {
+__device__ void encode_rows(const QTensor& q, float alpha, const QBatch& p, uint2* qbuf) {
   const T* x = static_cast<const T*>(q.x);
   const uint32_t kbpr = (uint32_t)(q.cols >> 4);
-  const uint64_t nblk = (uint64_t)q.rows * kbpr;
+  const uint32_t nblk = (uint32_t)q.rows * kbpr;  // < 2^32, checked on the host
+  const FastDiv div = make_fastdiv(kbpr);
   const bool fos = p.four_over_six != 0;
   const ScaleCtx ctx = make_scale_ctx(alpha);
-  for (uint64_t u = (uint64_t)blockIdx.x * kThreads + threadIdx.x; u < nblk;
-       u += (uint64_t)gridDim.x * kThreads) {
-    const uint32_t r = (uint32_t)u / kbpr, kb = (uint32_t)u - r * kbpr;
+  const uint32_t stride = gridDim.x * kThreads;
+  auto src = [&](uint32_t b) {
+    const uint32_t r = fastdiv(b, div);
+    return x + (int64_t)r * q.ld + (int64_t)(b - r * kbpr) * 16;
+  };
+  auto codes_at = [&](uint32_t b) {
+    const uint32_t r = fastdiv(b, div);
+    return q.codes + (int64_t)r * (q.cols >> 1) + (int64_t)(b - r * kbpr) * 8;
+  };
+  auto scale_at = [&](uint32_t b) {
+    const uint32_t r = fastdiv(b, div);
+    return q.scales + sf_offset(r, b - r * kbpr, kbpr, p.sf_layout);
+  };
+  auto redo = [&](uint2 it) {
+    RawBlock<T> blk;
+    blk.load(src(it.x));
     float v[16];
-    load16(x + (int64_t)r * q.ld + (int64_t)kb * 16, v);
+    blk.widen(v);
     if (RHT) rht16(v, p.mask);
-    uint32_t lo, hi, sc;
-    quantize_block16(v, ctx, fos, lo, hi, sc);
-    *reinterpret_cast<uint2*>(q.codes + (int64_t)r * (q.cols >> 1) + (int64_t)kb * 8) =
-        make_uint2(lo, hi);
-    q.scales[sf_offset(r, kb, kbpr, p.sf_layout)] = (uint8_t)sc;
+    redo_block(v, it.y, ctx, fos, codes_at(it.x), scale_at(it.x));
+  };
+  WarpQueue wq{qbuf, 0u};
+  uint32_t u = blockIdx.x * kThreads + threadIdx.x;
+  RawBlock<T> next;
+  if (u < nblk) next.load(src(u));
+  for (uint32_t base = blockIdx.x * kThreads; base < nblk; base += stride, u += stride) {
+    const RawBlock<T> cur = next;
+    if (u + stride < nblk) next.load(src(u + stride));
+    uint32_t st = kBlockDone, sc = 0u;
+    if (u < nblk) {
+      float v[16];
+      cur.widen(v);
+      if (RHT) rht16(v, p.mask);
+      uint32_t lo, hi;
+      st = quantize_block16_try(v, ctx, fos, lo, hi, sc);
+      if (st == kBlockDone) store_codes(codes_at(u), lo, hi);
+      if (st != kBlockExact) *scale_at(u) = (uint8_t)sc;
+    }
+    wq.push(st != kBlockDone, u, st == kBlockExact ? kRedoAll : sc);
+    if (wq.n > kQueueCap - 32) wq.drain(redo);
   }
+  wq.drain(redo);
   if (p.sf_layout == 1) zero_sf_padding(q.scales, q.rows, kbpr);
 }
 
 // Encode pass, blocks along rows; output transposed: codes [cols, rows/2],
-// scales for cols rows x rows/16 blocks.  Unit = column pair x 64 rows.
+// scales for cols rows x rows/16 blocks.  Unit = column pair x 16 rows (two
+// blocks), the next unit's loads issued before the current one is encoded.
 template <typename T, bool RHT>
-__device__ void encode_cols(const QTensor& q, float alpha, const QBatch& p) {
+__device__ void encode_cols(const QTensor& q, float alpha, const QBatch& p, uint2* qbuf) {
   const T* x = static_cast<const T*>(q.x);
-  const uint32_t ncp = (uint32_t)((q.cols + 1) >> 1);
-  const uint32_t nrc = (uint32_t)((q.rows + 63) >> 6);
-  const uint64_t nunits = (uint64_t)ncp * nrc;
+  const uint32_t ncp = (uint32_t)(q.cols >> 1);
+  const uint32_t kb_total = (uint32_t)(q.rows >> 4);
+  const uint32_t nunits = ncp * kb_total;
   const int64_t out_row_bytes = q.rows >> 1;
-  const int64_t kb_total = q.rows >> 4;
+  const FastDiv div = make_fastdiv(ncp), div_out = make_fastdiv(kb_total);
   const bool fos = p.four_over_six != 0;
   const ScaleCtx ctx = make_scale_ctx(alpha);
-  for (uint64_t u = (uint64_t)blockIdx.x * kThreads + threadIdx.x; u < nunits;
-       u += (uint64_t)gridDim.x * kThreads) {
-    const uint32_t rc = (uint32_t)u / ncp, cp = (uint32_t)u - rc * ncp;
-    const int64_t c0 = 2 * (int64_t)cp;
-#pragma unroll 1
-    for (int g = 0; g < 4; ++g) {
-      const int64_t rg = 64 * (int64_t)rc + 16 * g;
-      if (rg >= q.rows) break;
-      float a[16], b[16];
+  const uint32_t stride = gridDim.x * kThreads;
+  auto src = [&](uint32_t unit) {
+    const uint32_t rg = fastdiv(unit, div);
+    return x + (int64_t)rg * 16 * q.ld + 2 * (int64_t)(unit - rg * ncp);
+  };
+  // queued entries hold the output block index c * kb_total + kb
+  auto redo = [&](uint2 it) {
+    const uint32_t c = fastdiv(it.x, div_out), kb = it.x - c * kb_total;
+    float v[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) load2(x + (rg + j) * q.ld + c0, a[j], b[j]);
-      if (RHT) {
-        rht16(a, p.mask);
-        rht16(b, p.mask);
+    for (int j = 0; j < 16; ++j) v[j] = load1(x + ((int64_t)kb * 16 + j) * q.ld + c);
+    if (RHT) rht16(v, p.mask);
+    redo_block(v, it.y, ctx, fos, q.codes + (int64_t)c * out_row_bytes + (int64_t)kb * 8,
+               q.scales + sf_offset(c, kb, kb_total, p.sf_layout));
+  };
+  WarpQueue wq{qbuf, 0u};
+  uint32_t u = blockIdx.x * kThreads + threadIdx.x;
+  RawPair<T> next;
+  if (u < nunits) next.load(src(u), q.ld);
+  for (uint32_t base = blockIdx.x * kThreads; base < nunits; base += stride, u += stride) {
+    const RawPair<T> cur = next;
+    if (u + stride < nunits) next.load(src(u + stride), q.ld);
+    uint32_t st[2] = {kBlockDone, kBlockDone}, sc[2] = {0u, 0u}, ob[2] = {0u, 0u};
+    if (u < nunits) {
+      const uint32_t kb = fastdiv(u, div), c0 = 2 * (u - kb * ncp);
+      float col[2][16];
+      cur.widen(col[0], col[1]);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (RHT) rht16(col[h], p.mask);
+        uint32_t lo, hi;
+        st[h] = quantize_block16_try(col[h], ctx, fos, lo, hi, sc[h]);
+        const uint32_t c = c0 + h;
+        ob[h] = c * kb_total + kb;
+        if (st[h] == kBlockDone)
+          store_codes(q.codes + (int64_t)c * out_row_bytes + (int64_t)kb * 8, lo, hi);
+        if (st[h] != kBlockExact) q.scales[sf_offset(c, kb, kb_total, p.sf_layout)] = (uint8_t)sc[h];
       }
-      uint32_t lo, hi, sc;
-      quantize_block16(a, ctx, fos, lo, hi, sc);
-      *reinterpret_cast<uint2*>(q.codes + c0 * out_row_bytes + (rg >> 1)) = make_uint2(lo, hi);
-      q.scales[sf_offset(c0, rg >> 4, kb_total, p.sf_layout)] = (uint8_t)sc;
-      quantize_block16(b, ctx, fos, lo, hi, sc);
-      *reinterpret_cast<uint2*>(q.codes + (c0 + 1) * out_row_bytes + (rg >> 1)) =
-          make_uint2(lo, hi);
-      q.scales[sf_offset(c0 + 1, rg >> 4, kb_total, p.sf_layout)] = (uint8_t)sc;
     }
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      wq.push(st[h] != kBlockDone, ob[h], st[h] == kBlockExact ? kRedoAll : sc[h]);
+    if (wq.n > kQueueCap - 64) wq.drain(redo);
   }
+  wq.drain(redo);
   if (p.sf_layout == 1) zero_sf_padding(q.scales, q.cols, kb_total);
 }
 
 // Encode pass, 16x16 tiles.  A warp holds two adjacent tiles of one 16-row
 // band: lane l owns row (l & 15) of tile (l >> 4).  Tile max and tile error
 // reduce across the 16 lanes of a half-warp with xor shuffles 8, 4, 2, 1 --
-// the same pairwise order as the per-row sum.
+// the same pairwise order as the per-row sum, and the same result on every
+// lane of the half-warp, so each tile's decisions are uniform over its lanes.
+// The pick is certified from approximate row errors as in the 1D path (the
+// tile margin is the sum of its 16 rows' margins); a tile too close to call
+// is redone exactly by its half-warp, and rows whose codes are ambiguous are
+// queued for an exact redo under the tile's scale.
 template <typename T>
-__device__ void encode_2d(const QTensor& q, float alpha, const QBatch& p) {
+__device__ void encode_2d(const QTensor& q, float alpha, const QBatch& p, uint2* qbuf) {
   const T* x = static_cast<const T*>(q.x);
   const uint32_t kbpr = (uint32_t)(q.cols >> 4);
   const uint32_t npair = (kbpr + 1) >> 1;
   const uint32_t nunits = (uint32_t)(q.rows >> 4) * npair;
   const int lane = threadIdx.x & 31;
+  const unsigned hmask = 0xFFFFu << (lane & 16);
   const uint32_t warps = kThreads / 32;
   const bool fos = p.four_over_six != 0;
   const ScaleCtx ctx = make_scale_ctx(alpha);
+  const FastDiv div = make_fastdiv(npair), div_blk = make_fastdiv(kbpr);
+  // queued entries hold the block index r * kbpr + kb and the tile's scale
+  auto redo = [&](uint2 it) {
+    const uint32_t r = fastdiv(it.x, div_blk), kb = it.x - r * kbpr;
+    float v[16];
+    load16(x + (int64_t)r * q.ld + (int64_t)kb * 16, v);
+    redo_block(v, it.y, ctx, fos, q.codes + (int64_t)r * (q.cols >> 1) + (int64_t)kb * 8, nullptr);
+  };
+  WarpQueue wq{qbuf, 0u};
   for (uint32_t u = blockIdx.x * warps + (threadIdx.x >> 5); u < nunits; u += gridDim.x * warps) {
-    const uint32_t tr = u / npair, tp = u - tr * npair;
+    const uint32_t tr = fastdiv(u, div), tp = u - tr * npair;
     const int64_t r = (int64_t)tr * 16 + (lane & 15);
     const uint32_t kb = tp * 2 + (lane >> 4);
     const bool valid = kb < kbpr;
@@ -263,27 +466,56 @@ __device__ void encode_2d(const QTensor& q, float alpha, const QBatch& p) {
     for (int o = 8; o > 0; o >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xFFFFFFFFu, tmax, o));
     uint32_t e6, e4;
     scale_codes(tmax, ctx, e6, e4);
-    Cand c6 = encode16(v, cand_scale(e6, alpha));
-    float err6 = c6.err;
+    const float s6 = cand_scale(e6, alpha);
+    uint32_t ew = e6, lo = 0u, hi = 0u, st = kBlockDone;
+    float sw = s6;
+    bool exact_tile = false;
+    if (fos && e4 != e6) {
+      const float s4 = cand_scale(e4, alpha);
+      int pick = 2;
+      if (fast_pick_ok(e6, s6, s4)) {
+        float a6 = approx_err16(v, rcp_approx(s6)), a4 = approx_err16(v, rcp_approx(s4));
 #pragma unroll
-    for (int o = 8; o > 0; o >>= 1) err6 = __fadd_rn(err6, __shfl_xor_sync(0xFFFFFFFFu, err6, o));
-    uint32_t lo = c6.lo, hi = c6.hi, sc = e6;
-    if (fos) {
-      Cand c4 = encode16(v, cand_scale(e4, alpha));
-      float err4 = c4.err;
+        for (int o = 8; o > 0; o >>= 1) {
+          a6 += __shfl_xor_sync(hmask, a6, o);
+          a4 += __shfl_xor_sync(hmask, a4, o);
+        }
+        pick = certified_pick(a6, s6, a4, s4, 16.0f * kPickMargin);
+      }
+      if (pick == 1) {
+        ew = e4;
+        sw = s4;
+      } else if (pick == 2) {  // exact tile errors
+        exact_tile = true;
+        Cand c6 = encode16(v, s6);
+        Cand c4 = encode16(v, s4);
+        float err6 = c6.err, err4 = c4.err;
 #pragma unroll
-      for (int o = 8; o > 0; o >>= 1) err4 = __fadd_rn(err4, __shfl_xor_sync(0xFFFFFFFFu, err4, o));
-      if (err4 < err6) {
-        lo = c4.lo;
-        hi = c4.hi;
-        sc = e4;
+        for (int o = 8; o > 0; o >>= 1) {
+          err6 = __fadd_rn(err6, __shfl_xor_sync(hmask, err6, o));
+          err4 = __fadd_rn(err4, __shfl_xor_sync(hmask, err4, o));
+        }
+        const bool four = err4 < err6;
+        lo = four ? c4.lo : c6.lo;
+        hi = four ? c4.hi : c6.hi;
+        ew = four ? e4 : e6;
       }
     }
-    if (valid) {
-      *reinterpret_cast<uint2*>(q.codes + r * (q.cols >> 1) + (int64_t)kb * 8) = make_uint2(lo, hi);
-      q.scales[sf_offset(r, kb, kbpr, p.sf_layout)] = (uint8_t)sc;
+    if (!exact_tile && sw != 0.0f) {
+      uint32_t w[2];
+      st = rcp_ok(sw) && codes16_try(v, rcp_approx(sw), w) ? kBlockDone : kBlockCodes;
+      lo = w[0];
+      hi = w[1];
     }
+    const uint32_t blk = (uint32_t)r * kbpr + kb;
+    if (valid) {
+      if (st == kBlockDone) store_codes(q.codes + r * (q.cols >> 1) + (int64_t)kb * 8, lo, hi);
+      q.scales[sf_offset(r, kb, kbpr, p.sf_layout)] = (uint8_t)ew;
+    }
+    wq.push(valid && st != kBlockDone, blk, ew);
+    if (wq.n > kQueueCap - 32) wq.drain(redo);
   }
+  wq.drain(redo);
   if (p.sf_layout == 1) zero_sf_padding(q.scales, q.rows, kbpr);
 }
 
@@ -312,8 +544,13 @@ __global__ void __launch_bounds__(kThreads) finalize_kernel(const __grid_constan
 
 // Encode pass over tensor blockIdx.y.  ga = number of amax partials (0 when
 // the global scale is given).
+// Resident CTAs per SM the encode kernels are compiled for: the row-axis mode
+// holds two 16-element columns per thread and needs the larger register file.
+template <int MODE>
+constexpr int encode_min_blocks() { return MODE == 1 ? 2 : 3; }
+
 template <typename T, int MODE, bool RHT>
-__global__ void __launch_bounds__(kThreads, 4) encode_kernel(const __grid_constant__ QBatch p, int ga) {
+__global__ void __launch_bounds__(kThreads, encode_min_blocks<MODE>()) encode_kernel(const __grid_constant__ QBatch p, int ga) {
   const int t = blockIdx.y;
   float alpha;
   if (p.gs_in) {
@@ -323,18 +560,20 @@ __global__ void __launch_bounds__(kThreads, 4) encode_kernel(const __grid_consta
     alpha = alpha_from_amax(reduce_partials(p.partials + t * kMaxAmaxCtas, ga));
   }
   if (blockIdx.x == 0 && threadIdx.x == 0 && p.t[t].gs_out) *p.t[t].gs_out = alpha;
-  if (MODE == kModeRows) encode_rows<T, RHT>(p.t[t], alpha, p);
-  else if (MODE == kModeCols) encode_cols<T, RHT>(p.t[t], alpha, p);
-  else encode_2d<T>(p.t[t], alpha, p);
+  __shared__ uint2 queue[kThreads / 32][kQueueCap];
+  uint2* qbuf = queue[threadIdx.x >> 5];
+  if (MODE == kModeRows) encode_rows<T, RHT>(p.t[t], alpha, p, qbuf);
+  else if (MODE == kModeCols) encode_cols<T, RHT>(p.t[t], alpha, p, qbuf);
+  else encode_2d<T>(p.t[t], alpha, p, qbuf);
 }
 
 uint64_t max_units(const QBatch& b, int mode) {
   uint64_t units = 0;
   for (int i = 0; i < b.n; ++i) {
     const QTensor& q = b.t[i];
-    // 16-blocks (rows), column pairs x 64 rows (cols), threads of 2-tile warps (2D)
+    // 16-blocks (rows), column pairs x 16 rows (cols), threads of 2-tile warps (2D)
     uint64_t u = mode == kModeRows ? (uint64_t)q.rows * (uint64_t)(q.cols / 16)
-               : mode == kModeCols ? (uint64_t)((q.cols + 1) / 2) * (uint64_t)((q.rows + 63) / 64)
+               : mode == kModeCols ? (uint64_t)(q.cols / 2) * (uint64_t)(q.rows / 16)
                                    : (uint64_t)(q.rows / 16) * (uint64_t)((q.cols / 16 + 1) / 2) * 32;
     units = u > units ? u : units;
   }
@@ -426,13 +665,13 @@ int grid_for(uint64_t work_items, int n_tensors) {
 }  // namespace
 
 int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
+  static const int n = [] {
+    int dev = 0, c = 0;
     cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-  }
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0)
+      c = 148;
+    return c;
+  }();
   return n;
 }
 
@@ -468,7 +707,16 @@ cudaError_t launch_mode(const QBatch& b, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     if (b.amax_only) return launch_ex(finalize_kernel, dim3(b.n), s, true, b, ga);
   }
-  uint64_t cap = (uint64_t)num_sms() * 4 / (uint64_t)b.n;
+  // one full wave of resident CTAs across all tensors
+  static const int occ = [] {
+    int o = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, encode_kernel<T, MODE, RHT>, kThreads,
+                                                      0) != cudaSuccess ||
+        o < 1)
+      o = encode_min_blocks<MODE>();
+    return o;
+  }();
+  uint64_t cap = (uint64_t)num_sms() * (uint64_t)occ / (uint64_t)b.n;
   if (cap < 1) cap = 1;
   uint64_t want = (units + per_cta - 1) / per_cta;
   const unsigned gx = (unsigned)(want < 1 ? 1 : (want < cap ? want : cap));
