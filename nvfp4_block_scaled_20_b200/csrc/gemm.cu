@@ -5,21 +5,26 @@
 // A [M, K] and B [N, K] are packed E2M1 codes (K-major), sA / sB are UE4M3
 // scales in the tcgen05 block-scaled layout.  Persistent kernel: one CTA per
 // SM walks 128 x 256 output tiles in a grouped (L2-friendly) order.
-//   warp 0      TMA producer: codes with cp.async.bulk.tensor (128B swizzle),
-//               scale atoms with cp.async.bulk, into a 4-deep ring that runs
-//               ahead across tile boundaries;
-//   warp 1      allocates tensor memory; one thread issues, per MMA k-block,
-//               the tcgen05.cp of its scale atoms into a 12-column slot and
-//               the tcgen05.mma kind::mxf4nvf4 (block16 scales, K = 64);
-//               tcgen05.commit releases ring stages and signals accumulators;
-//   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulator (two warps per
-//               32-lane quadrant, half of the columns each), x alpha_a*alpha_b,
-//               optional GELU(tanh), bf16 / fp32 stores.
-// Tensor memory holds two 256-column accumulators and one MMA k-block's scale
-// factors (12 columns): 524 of the 512 columns, so the second accumulator
-// starts at column 240 and the two share 16 columns.  The epilogue drains the
-// shared columns first and releases them, so the next tile's MMAs wait only
-// for that, not for the whole drain.
+//   warp 0       TMA producer: codes with cp.async.bulk.tensor (128B swizzle),
+//                scale atoms with cp.async.bulk, into a 4-deep ring that runs
+//                ahead across tile boundaries;
+//   warp 1       allocates tensor memory; one thread issues the four
+//                tcgen05.mma kind::mxf4nvf4 (block16 scales, K = 64) of each
+//                stage; tcgen05.commit releases ring stages and scale slots
+//                and signals accumulators;
+//   warps 2..9   epilogue: tcgen05.ld of the fp32 accumulator (two warps per
+//                32-lane quadrant, half of the columns each), x alpha_a*alpha_b,
+//                optional GELU(tanh), bf16 / fp32 stores;
+//   warps 10..13 scale staging, one per 32-lane quadrant: each stage's scale
+//                atoms from shared memory into registers, then tcgen05.st into
+//                one of two 48-column scale slots of tensor memory, in the
+//                layout the MMA reads (every quadrant holds all four 32-row
+//                groups' scales).  Writing scales from these warps keeps the
+//                MMA thread's in-order tcgen05 queue free of scale copies.
+// Tensor memory: accumulator 0 at columns [0, 256), accumulator 1 at
+// [160, 416) -- the two share 96 columns, which the epilogue drains first and
+// releases so the next tile's MMAs wait only for that -- and the two scale
+// slots at [416, 512).
 // Every wait is bounded (wall clock through %globaltimer); on a timeout the
 // CTA records NVFP4_ERR_TIMEOUT in the device error word, drains what it
 // issued and frees its tensor memory before returning.
@@ -39,7 +44,9 @@ constexpr int BK_BYTES = BK / 2;  // one 128-byte swizzle row
 constexpr int MMA_K = 64;         // K per tcgen05.mma (kind::mxf4nvf4)
 constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;
-constexpr int kNumThreads = (2 + kEpiWarps) * 32;
+constexpr int kSfWarps = 4;
+constexpr int kSfWarp0 = 2 + kEpiWarps;  // first scale-staging warp
+constexpr int kNumThreads = (2 + kEpiWarps + kSfWarps) * 32;
 constexpr int kABytes = BM * BK_BYTES;          // 16 KB
 constexpr int kBBytes = BN * BK_BYTES;          // 32 KB
 constexpr int kSfaBytes = 4 * 512;              // 4 atoms (128 rows x 16 blocks)
@@ -48,10 +55,11 @@ constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
 // tensor memory columns
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAcc1Col = 240;   // accumulator 0 at column 0, 1 at 240
-constexpr uint32_t kOvlCols = 16;    // columns [240, 256) belong to both
-constexpr uint32_t kSfaCol = 496;    // 4 columns: one MMA k-block of A scales
-constexpr uint32_t kSfbCol = 500;    // 8 columns: one MMA k-block of B scales
+constexpr uint32_t kAcc1Col = 160;   // accumulator 0 at column 0, 1 at 160
+constexpr uint32_t kOvlCols = 96;    // columns [160, 256) belong to both
+constexpr uint32_t kSfSlotCol = 416; // two scale slots of 48 columns
+constexpr uint32_t kSfSlotCols = 48; // A: 4 per MMA k-block (16), B: 8 per k-block (32)
+constexpr int kSfSlots = 2;
 constexpr int kGroupM = 8;           // tile raster: 8 M-tiles per group
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s when draining after an abort
@@ -124,10 +132,6 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                    bar)
                : "memory");
 }
-__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
-}
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
                                        uint32_t accumulate) {
@@ -150,6 +154,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t r[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Tensor-memory stores of 16 / 32 consecutive 32-bit columns for the 32 lanes
+// of this warp's quadrant (taddr carries the quadrant's first lane).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t r[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // Shared-memory matrix descriptor (tcgen05 format): start address >> 4 in
 // bits 0-13, leading byte offset >> 4 in 16-29, stride byte offset >> 4 in
 // 32-45, version 1 in 46-47, base offset 0, layout type in 61-63.
@@ -162,11 +180,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 // 1024 bytes apart.
 __device__ __forceinline__ uint64_t operand_desc(uint32_t addr) {
   return smem_desc(addr, 16, 1024, 2 /*SWIZZLE_128B*/);
-}
-// Scale atom source for tcgen05.cp 32x128b: 32 rows x 16 bytes, contiguous
-// (8-row core matrices 128 bytes apart, no swizzle).
-__device__ __forceinline__ uint64_t sf_desc(uint32_t addr) {
-  return smem_desc(addr, 0, 128, 0 /*SWIZZLE_NONE*/);
 }
 // Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (format 1), UE4M3
 // scales (bit 23 = 0), K-major A and B, N >> 3 in bits 17-22, M >> 4 in
@@ -241,13 +254,15 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   uint8_t* sSFA = sB + kStages * kBBytes;
   uint8_t* sSFB = sSFA + kStages * kSfaBytes;
   uint64_t* bars = (uint64_t*)(sSFB + kStages * kSfbBytes);
-  uint64_t* full = bars;                        // [kStages]   TMA -> MMA
-  uint64_t* empty = bars + kStages;             // [kStages]   MMA -> TMA
-  uint64_t* acc_full = bars + 2 * kStages;      // [2]         MMA -> epilogue
-  uint64_t* acc_empty = bars + 2 * kStages + 2; // [2]         epilogue -> MMA
-  uint64_t* ovl_free = bars + 2 * kStages + 4;  // [1]         shared columns drained
-  uint64_t* mma_done = bars + 2 * kStages + 5;  // [1]         all MMAs of this CTA done
-  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * kStages + 6);
+  uint64_t* full = bars;                         // [kStages]  TMA -> MMA, scale warps
+  uint64_t* empty = bars + kStages;              // [kStages]  MMA + scale warps -> TMA
+  uint64_t* sf_full = bars + 2 * kStages;        // [2]        scale warps -> MMA
+  uint64_t* sf_empty = sf_full + kSfSlots;       // [2]        MMA -> scale warps
+  uint64_t* acc_full = sf_empty + kSfSlots;      // [2]        MMA -> epilogue
+  uint64_t* acc_empty = acc_full + 2;            // [2]        epilogue -> MMA
+  uint64_t* ovl_free = acc_empty + 2;            // [1]        shared columns drained
+  uint64_t* mma_done = ovl_free + 1;             // [1]        all MMAs of this CTA done
+  uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -260,13 +275,17 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&empty[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1 + kSfWarps);
+    }
+    for (int b = 0; b < kSfSlots; ++b) {
+      mbar_init(smem_u32(&sf_full[b]), kSfWarps);
+      mbar_init(smem_u32(&sf_empty[b]), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&acc_full[b]), 1);
       mbar_init(smem_u32(&acc_empty[b]), kEpiWarps);
     }
-    mbar_init(smem_u32(ovl_free), kEpiWarps / 2);
+    mbar_init(smem_u32(ovl_free), kEpiWarps);
     mbar_init(smem_u32(mma_done), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -330,7 +349,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = instr_desc(BM, BN);
-      const uint32_t t_sfa = tmem + kSfaCol, t_sfb = tmem + kSfbCol;
       uint32_t it = 0, tile_i = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++tile_i) {
@@ -349,7 +367,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const uint32_t t_acc = tmem + (b ? kAcc1Col : 0u);
         for (int kt = 0; kt < num_kt; ++kt, ++it) {
           const int s = it % kStages;
-          if (!mbar_wait(smem_u32(&full[s]), (it / kStages) & 1u, abort_flag, kWaitLimitNs)) {
+          const uint32_t slot = it % kSfSlots;
+          if (!mbar_wait(smem_u32(&full[s]), (it / kStages) & 1u, abort_flag, kWaitLimitNs) ||
+              !mbar_wait(smem_u32(&sf_full[slot]), (it / kSfSlots) & 1u, abort_flag, kWaitLimitNs)) {
             ok = false;
             break;
           }
@@ -357,18 +377,12 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           const int nmma = min(4, (p.K - kt * BK) / MMA_K);
           const uint32_t a_base = smem_u32(sA + s * kABytes);
           const uint32_t b_base = smem_u32(sB + s * kBBytes);
-          const uint32_t sfa_base = smem_u32(sSFA + s * kSfaBytes);
-          const uint32_t sfb_base = smem_u32(sSFB + s * kSfbBytes);
-          for (int k = 0; k < nmma; ++k) {
-            // tcgen05 operations from one thread execute in issue order: the
-            // copy into the scale slot waits for the previous MMA's reads
-            tc_cp_sf(t_sfa, sf_desc(sfa_base + 512 * k));
-            tc_cp_sf(t_sfb, sf_desc(sfb_base + 512 * k));
-            tc_cp_sf(t_sfb + 4, sf_desc(sfb_base + 2048 + 512 * k));
-            tc_mma(t_acc, operand_desc(a_base + 32 * k), operand_desc(b_base + 32 * k), idesc, t_sfa,
-                   t_sfb, (kt > 0 || k > 0) ? 1u : 0u);
-          }
+          const uint32_t t_sf = tmem + kSfSlotCol + slot * kSfSlotCols;
+          for (int k = 0; k < nmma; ++k)
+            tc_mma(t_acc, operand_desc(a_base + 32 * k), operand_desc(b_base + 32 * k), idesc,
+                   t_sf + 4 * k, t_sf + 16 + 8 * k, (kt > 0 || k > 0) ? 1u : 0u);
           tc_commit(smem_u32(&empty[s]));
+          tc_commit(smem_u32(&sf_empty[slot]));
         }
         // signals once this tile's MMAs (and everything before) completed
         tc_commit(smem_u32(&acc_full[b]));
@@ -381,11 +395,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       tc_commit(smem_u32(mma_done));
       mbar_wait(smem_u32(mma_done), 0, nullptr, kWaitLimitNs);
     }
-  } else {
+  } else if (warp < kSfWarp0) {
     // ------------------------------------------------------------ epilogue
     const int e = warp - 2;        // 0..7
     const int quad = warp & 3;     // TMEM lanes 32*quad .. 32*quad+31
-    const int half = e >> 2;       // columns [128*half, 128*half + 128)
+    const int half = e >> 2;       // 0 / 1: first / second half of each column range
     const float scale = __fmul_rn(*p.a_alpha, *p.b_alpha);
     uint32_t tile_i = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tile_i) {
@@ -402,34 +416,79 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       const uint32_t t_acc = tmem + (b ? kAcc1Col : 0u) + ((uint32_t)(quad * 32) << 16);
       const int row = m0 + quad * 32 + lane;
       const bool quad_live = m0 + quad * 32 < p.M;  // warp-uniform
-      // the 16 columns shared with the other accumulator: tile columns
-      // 240..255 of accumulator 0, 0..15 of accumulator 1
-      const int ovl_half = b ? 0 : 1;
+      // The columns shared with the other accumulator (tile columns 160..255
+      // of accumulator 0, 0..95 of accumulator 1) go first, split between
+      // the two warps of each quadrant; then the rest.
       const int ovl_c0 = b ? 0 : 256 - (int)kOvlCols;
-      if (half == ovl_half) {
+      const int rest_c0 = b ? (int)kOvlCols : 0;
+      constexpr int kOvlPer = (int)kOvlCols / 2, kRestPer = (256 - (int)kOvlCols) / 2;
+      auto drain = [&](int c0, int ncols) {
 #pragma unroll 1
-        for (int c = ovl_c0; c < ovl_c0 + (int)kOvlCols; c += 16) {
+        for (int c = c0; c < c0 + ncols; c += 16) {
           if (!quad_live || n0 + c >= p.N) continue;
           uint32_t r[16];
           tmem_ld16(t_acc + (uint32_t)c, r);
           if (row < p.M) store16(p, row, n0 + c, r, scale);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(ovl_free));
-      }
-#pragma unroll 1
-      for (int j = 0; j < 8; ++j) {
-        const int c = half * 128 + j * 16;
-        if (half == ovl_half && c >= ovl_c0 && c < ovl_c0 + (int)kOvlCols) continue;
-        if (!quad_live || n0 + c >= p.N) continue;
-        uint32_t r[16];
-        tmem_ld16(t_acc + (uint32_t)c, r);
-        if (row < p.M) store16(p, row, n0 + c, r, scale);
-      }
+      };
+      drain(ovl_c0 + half * kOvlPer, kOvlPer);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(ovl_free));
+      drain(rest_c0 + half * kRestPer, kRestPer);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
+    }
+  } else {
+    // ------------------------------------------------------------ scale staging
+    // Quadrant q's lanes get, per MMA k-block k of the stage: A columns
+    // 4k + j = word j of row (lane) of the k-block's A atom (the four 32-row
+    // groups' 4 scales each), B columns 16 + 8k + 4h + j = word j of row
+    // (lane) of band h's atom.
+    const int quad = warp & 3;
+    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int kt = 0; kt < num_kt; ++kt, ++it) {
+        const int s = it % kStages;
+        const uint32_t slot = it % kSfSlots;
+        if (!mbar_wait(smem_u32(&full[s]), (it / kStages) & 1u, abort_flag, kWaitLimitNs) ||
+            !mbar_wait(smem_u32(&sf_empty[slot]), ((it / kSfSlots) & 1u) ^ 1u, abort_flag,
+                       kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t ra[16], rb[32];
+        const uint8_t* sfa = sSFA + s * kSfaBytes + 16 * lane;
+        const uint8_t* sfb = sSFB + s * kSfbBytes + 16 * lane;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint4 a4 = *reinterpret_cast<const uint4*>(sfa + 512 * k);
+          const uint4 b0 = *reinterpret_cast<const uint4*>(sfb + 512 * k);
+          const uint4 b1 = *reinterpret_cast<const uint4*>(sfb + 2048 + 512 * k);
+          ra[4 * k] = a4.x, ra[4 * k + 1] = a4.y, ra[4 * k + 2] = a4.z, ra[4 * k + 3] = a4.w;
+          rb[8 * k] = b0.x, rb[8 * k + 1] = b0.y, rb[8 * k + 2] = b0.z, rb[8 * k + 3] = b0.w;
+          rb[8 * k + 4] = b1.x, rb[8 * k + 5] = b1.y, rb[8 * k + 6] = b1.z, rb[8 * k + 7] = b1.w;
+        }
+        // the stage's scale bytes are in registers: the ring slot may refill
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
+        const uint32_t t_sf = tmem + lane_addr + kSfSlotCol + slot * kSfSlotCols;
+        tmem_st16(t_sf, ra);
+        tmem_st16(t_sf + 16, rb);
+        tmem_st16(t_sf + 32, rb + 16);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sf_full[slot]));
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      if (lane == 0) atomicOr(p.err, kDevErrTimeout);
     }
   }
 
