@@ -3,28 +3,35 @@
 //   out[m, n] = epi(alpha_a * alpha_b * sum_k a_mk * sA[m, k/16] * b_nk * sB[n, k/16])
 //
 // A [M, K] and B [N, K] are packed E2M1 codes (K-major), sA / sB are UE4M3
-// scales in the tcgen05 block-scaled layout.  Persistent kernel: one CTA per
-// SM walks 128 x 256 output tiles in a grouped (L2-friendly) order.
-//   warp 0       TMA producer: codes with cp.async.bulk.tensor (128B swizzle),
-//                scale atoms with cp.async.bulk, into a 4-deep ring that runs
-//                ahead across tile boundaries;
-//   warp 1       allocates tensor memory; one thread issues the four
-//                tcgen05.mma kind::mxf4nvf4 (block16 scales, K = 64) of each
-//                stage; tcgen05.commit releases ring stages and scale slots
-//                and signals accumulators;
-//   warps 2..9   epilogue: tcgen05.ld of the fp32 accumulator (two warps per
-//                32-lane quadrant, half of the columns each), x alpha_a*alpha_b,
+// scales in the tcgen05 block-scaled layout.  Persistent kernel of CTA pairs
+// (clusters of two on neighbouring SMs): each pair walks 256 x 256 output
+// tiles in a grouped (L2-friendly) order with 2-SM MMAs
+// (tcgen05.mma.cta_group::2, M = 256): CTA r of the pair holds A rows
+// [128 r, 128 r + 128) and B rows [128 r, 128 r + 128) of the tile in shared
+// memory and output rows [128 r, 128 r + 128) in tensor memory, so each SM
+// stores and serves only half of B -- the operand traffic through shared
+// memory per MMA is two thirds of a single-SM 128 x 256 tile's.
+//   warp 0       TMA producer (both CTAs): codes with the 2-SM form of
+//                cp.async.bulk.tensor (no multicast; completion counted on
+//                the leader CTA's barrier), scale atoms with cp.async.bulk
+//                into its own CTA, a 5-deep ring that runs ahead across tiles;
+//   warp 1       allocates tensor memory (cta_group::2); in the leader CTA one
+//                thread issues the four MMAs (kind::mxf4nvf4, block16 scales,
+//                K = 64) of each stage; tcgen05.commit multicast to both CTAs
+//                releases ring stages and scale slots and signals accumulators;
+//   warps 2..9   epilogue (both CTAs): tcgen05.ld of the CTA's 128 accumulator
+//                rows (two warps per 32-lane quadrant), x alpha_a*alpha_b,
 //                optional GELU(tanh), bf16 / fp32 stores;
-//   warps 10..13 scale staging, one per 32-lane quadrant: each stage's scale
-//                atoms from shared memory into registers, then tcgen05.st into
-//                one of two 48-column scale slots of tensor memory, in the
+//   warps 10..13 scale staging, one per 32-lane quadrant (both CTAs): each
+//                stage's scale atoms from shared memory into registers, then
+//                tcgen05.st into one of two 48-column scale slots, in the
 //                layout the MMA reads (every quadrant holds all four 32-row
-//                groups' scales).  Writing scales from these warps keeps the
-//                MMA thread's in-order tcgen05 queue free of scale copies.
-// Tensor memory: accumulator 0 at columns [0, 256), accumulator 1 at
-// [160, 416) -- the two share 96 columns, which the epilogue drains first and
-// releases so the next tile's MMAs wait only for that -- and the two scale
-// slots at [416, 512).
+//                groups' scales; B scales for all 256 tile columns in each
+//                CTA).  Keeping scale copies out of the MMA thread's in-order
+//                tcgen05 queue lets the MMAs run back to back.
+// Tensor memory (each CTA): accumulator 0 at columns [0, 256), accumulator 1
+// at [160, 416) -- the two share 96 columns, which the epilogue drains first
+// and releases -- and the two scale slots at [416, 512).
 // Every wait is bounded (wall clock through %globaltimer); on a timeout the
 // CTA records NVFP4_ERR_TIMEOUT in the device error word, drains what it
 // issued and frees its tensor memory before returning.
@@ -37,22 +44,22 @@ namespace nvfp4 {
 
 namespace {
 
-constexpr int BM = 128;           // rows per tile (one TMEM lane per row)
-constexpr int BN = 256;           // columns per tile
+constexpr int BM = 128;           // rows per CTA (one TMEM lane per row); 256 per pair
+constexpr int BN = 256;           // columns per tile; each CTA holds half of B
 constexpr int BK = 256;           // K elements per stage = 128 bytes of codes per row
 constexpr int BK_BYTES = BK / 2;  // one 128-byte swizzle row
 constexpr int MMA_K = 64;         // K per tcgen05.mma (kind::mxf4nvf4)
-constexpr int kStages = 4;
+constexpr int kStages = 5;
 constexpr int kEpiWarps = 8;
 constexpr int kSfWarps = 4;
 constexpr int kSfWarp0 = 2 + kEpiWarps;  // first scale-staging warp
 constexpr int kNumThreads = (2 + kEpiWarps + kSfWarps) * 32;
-constexpr int kABytes = BM * BK_BYTES;          // 16 KB
-constexpr int kBBytes = BN * BK_BYTES;          // 32 KB
+constexpr int kABytes = BM * BK_BYTES;          // 16 KB: this CTA's A rows
+constexpr int kBBytes = (BN / 2) * BK_BYTES;    // 16 KB: this CTA's half of B
 constexpr int kSfaBytes = 4 * 512;              // 4 atoms (128 rows x 16 blocks)
-constexpr int kSfbBytes = (BN / 128) * 4 * 512;
+constexpr int kSfbBytes = (BN / 128) * 4 * 512; // both 128-row bands of the tile
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 512 /*barriers*/;
 // tensor memory columns
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAcc1Col = 160;   // accumulator 0 at column 0, 1 at 160
@@ -68,6 +75,21 @@ constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s when draining after a
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -80,8 +102,26 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
+// Arrive on a barrier of this CTA (release at CTA scope: prior shared-memory
+// reads are complete before the stage can be refilled).
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// Arrive on the leader CTA's copy of a barrier.  Only tensor-memory work is
+// handed over this way (scale slots written, accumulator columns read), and
+// that is ordered by tcgen05.fence::before_thread_sync on this side and
+// tcgen05.fence::after_thread_sync on the waiting side, so the arrive itself
+// is relaxed: a release at cluster scope would wait for this CTA's
+// outstanding global stores and bulk copies, hundreds of nanoseconds.
+__device__ __forceinline__ void mbar_arrive_leader(uint32_t local_bar, bool leader) {
+  if (leader) {
+    mbar_arrive(local_bar);
+  } else {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(remote) : "r"(local_bar));
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote)
+                 : "memory");
+  }
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -105,12 +145,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
   }
 }
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t c0,
-                                            int32_t c1, uint32_t bar) {
+// Tile load into this CTA's shared memory, completion counted on a barrier of
+// either CTA of the pair (2-SM form, no multicast).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int32_t c0,
+                                                 int32_t c1, uint32_t cluster_bar) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-      "%3}], [%4];" ::"r"(dst),
-      "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(bar)
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(cluster_bar)
       : "memory");
 }
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
@@ -127,17 +169,22 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
+// Arrives on the barrier at this shared-memory offset in both CTAs of the pair
+// once every tcgen05 operation issued so far by this thread has completed.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+      "[%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
 }
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                       uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                       uint32_t accumulate) {
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                            uint32_t accumulate) {
   asm volatile(
       "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
       "p; }" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
@@ -153,9 +200,8 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t r[16]) {
       : "memory");
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-
-// Tensor-memory stores of 16 / 32 consecutive 32-bit columns for the 32 lanes
-// of this warp's quadrant (taddr carries the quadrant's first lane).
+// Tensor-memory stores of 16 consecutive 32-bit columns for the 32 lanes of
+// this warp's quadrant (taddr carries the quadrant's first lane).
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t r[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
@@ -254,52 +300,59 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   uint8_t* sSFA = sB + kStages * kBBytes;
   uint8_t* sSFB = sSFA + kStages * kSfaBytes;
   uint64_t* bars = (uint64_t*)(sSFB + kStages * kSfbBytes);
-  uint64_t* full = bars;                         // [kStages]  TMA -> MMA, scale warps
-  uint64_t* empty = bars + kStages;              // [kStages]  MMA + scale warps -> TMA
-  uint64_t* sf_full = bars + 2 * kStages;        // [2]        scale warps -> MMA
-  uint64_t* sf_empty = sf_full + kSfSlots;       // [2]        MMA -> scale warps
-  uint64_t* acc_full = sf_empty + kSfSlots;      // [2]        MMA -> epilogue
-  uint64_t* acc_empty = acc_full + 2;            // [2]        epilogue -> MMA
-  uint64_t* ovl_free = acc_empty + 2;            // [1]        shared columns drained
-  uint64_t* mma_done = ovl_free + 1;             // [1]        all MMAs of this CTA done
+  uint64_t* full = bars;                      // [kStages] codes of both CTAs landed (leader)
+  uint64_t* sf_in = full + kStages;           // [kStages] this CTA's scale atoms landed
+  uint64_t* empty = sf_in + kStages;          // [kStages] stage free: MMAs done + scales read
+  uint64_t* sf_full = empty + kStages;        // [2] scale slot written by both CTAs (leader)
+  uint64_t* sf_empty = sf_full + kSfSlots;    // [2] scale slot's MMAs done
+  uint64_t* acc_full = sf_empty + kSfSlots;   // [2] accumulator complete
+  uint64_t* acc_empty = acc_full + 2;         // [2] accumulator drained by both CTAs (leader)
+  uint64_t* ovl_free = acc_empty + 2;         // [1] shared columns drained by both (leader)
+  uint64_t* mma_done = ovl_free + 1;          // [1] all MMAs of the pair done (leader)
   uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int num_m = (p.M + BM - 1) / BM, num_n = (p.N + BN - 1) / BN;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+  const int num_m = (p.M + 2 * BM - 1) / (2 * BM), num_n = (p.N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kt = (p.K + BK - 1) / BK;
   const int kgroups = p.K / 64;  // 4-block scale groups per 128-row band
-  const int nbands_total = (p.N + 127) / 128;
+  const int mbands_total = (p.M + 127) / 128, nbands_total = (p.N + 127) / 128;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&sf_in[s]), 1);
       mbar_init(smem_u32(&empty[s]), 1 + kSfWarps);
     }
     for (int b = 0; b < kSfSlots; ++b) {
-      mbar_init(smem_u32(&sf_full[b]), kSfWarps);
+      mbar_init(smem_u32(&sf_full[b]), 2 * kSfWarps);
       mbar_init(smem_u32(&sf_empty[b]), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&acc_full[b]), 1);
-      mbar_init(smem_u32(&acc_empty[b]), kEpiWarps);
+      mbar_init(smem_u32(&acc_empty[b]), 2 * kEpiWarps);
     }
-    mbar_init(smem_u32(ovl_free), kEpiWarps);
+    mbar_init(smem_u32(ovl_free), 2 * kEpiWarps);
     mbar_init(smem_u32(mma_done), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
                  "r"(kTmemCols)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
-  __syncthreads();
+  // both CTAs' barriers initialised and tensor memory allocated before any
+  // cross-CTA arrival
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // operands may be written by the preceding kernel (programmatic launch)
@@ -310,13 +363,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int t = pair; t < num_tiles && ok; t += num_pairs) {
         int mt, nt;
         tile_coords(t, num_m, num_n, mt, nt);
-        const int m0 = mt * BM, n0 = nt * BN;
-        int bands = 0;
-        for (int b = 0; b < BN / 128; ++b)
-          if (n0 / 128 + b < nbands_total) ++bands;
+        const int m0 = mt * 2 * BM + (int)rank * BM, nb0 = nt * BN + (int)rank * (BN / 2);
+        const int mband = mt * 2 + (int)rank;
         for (int kt = 0; kt < num_kt; ++kt, ++it) {
           const int s = it % kStages;
           const uint32_t round = it / kStages;
@@ -324,37 +375,46 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             ok = false;
             break;
           }
+          const uint32_t fb = map_to_rank(smem_u32(&full[s]), 0);
+          if (leader) mbar_expect_tx(smem_u32(&full[s]), 2 * (kABytes + kBBytes));
+          tma_load_2d_pair(smem_u32(sA + s * kABytes), &tmA, kt * BK_BYTES, m0, fb);
+          tma_load_2d_pair(smem_u32(sB + s * kBBytes), &tmB, kt * BK_BYTES, nb0, fb);
           const int atoms = min(4, kgroups - kt * 4);
-          const uint32_t bytes = kABytes + kBBytes + atoms * 512 * (1 + bands);
-          const uint32_t fb = smem_u32(&full[s]);
-          mbar_expect_tx(fb, bytes);
-          tma_load_2d(smem_u32(sA + s * kABytes), &tmA, kt * BK_BYTES, m0, fb);
-          tma_load_2d(smem_u32(sB + s * kBBytes), &tmB, kt * BK_BYTES, n0, fb);
-          bulk_load(smem_u32(sSFA + s * kSfaBytes),
-                    p.a_sf + ((int64_t)(m0 / 128) * kgroups + kt * 4) * 512, atoms * 512, fb);
-          for (int b = 0; b < bands; ++b)
-            bulk_load(smem_u32(sSFB + s * kSfbBytes + b * 2048),
-                      p.b_sf + ((int64_t)(n0 / 128 + b) * kgroups + kt * 4) * 512, atoms * 512, fb);
+          int nsf = mband < mbands_total ? 1 : 0;
+          for (int h = 0; h < 2; ++h) nsf += (nt * 2 + h < nbands_total) ? 1 : 0;
+          const uint32_t sb = smem_u32(&sf_in[s]);
+          mbar_expect_tx(sb, (uint32_t)(atoms * 512 * nsf));
+          if (mband < mbands_total)
+            bulk_load(smem_u32(sSFA + s * kSfaBytes),
+                      p.a_sf + ((int64_t)mband * kgroups + kt * 4) * 512, atoms * 512, sb);
+          for (int h = 0; h < 2; ++h)
+            if (nt * 2 + h < nbands_total)
+              bulk_load(smem_u32(sSFB + s * kSfbBytes + h * 2048),
+                        p.b_sf + ((int64_t)(nt * 2 + h) * kgroups + kt * 4) * 512, atoms * 512, sb);
         }
       }
       if (!ok) {
         *abort_flag = 1;
         atomicOr(p.err, kDevErrTimeout);
       }
-      // every stage issued must have landed before the CTA retires (bounded)
+      // every scale load issued must have landed before the CTA retires
+      // (the codes are waited for by the leader's MMA thread) -- bounded
       for (uint32_t j = (it > (uint32_t)kStages ? it - kStages : 0u); j < it; ++j)
-        mbar_wait(smem_u32(&full[j % kStages]), (j / kStages) & 1u, nullptr, kDrainLimitNs);
+        mbar_wait(smem_u32(&sf_in[j % kStages]), (j / kStages) & 1u, nullptr, kDrainLimitNs);
+      if (leader)
+        for (uint32_t j = (it > (uint32_t)kStages ? it - kStages : 0u); j < it; ++j)
+          mbar_wait(smem_u32(&full[j % kStages]), (j / kStages) & 1u, nullptr, kDrainLimitNs);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = instr_desc(BM, BN);
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = instr_desc(2 * BM, BN);
       uint32_t it = 0, tile_i = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++tile_i) {
+      for (int t = pair; t < num_tiles && ok; t += num_pairs, ++tile_i) {
         const uint32_t b = tile_i & 1u, use = tile_i >> 1;
-        // accumulator b drained by the epilogue of tile_i - 2, and the shared
-        // columns by the epilogue of tile_i - 1
+        // accumulator b drained by both CTAs' epilogues of tile_i - 2, and
+        // the shared columns by those of tile_i - 1
         if (use > 0 && !mbar_wait(smem_u32(&acc_empty[b]), (use - 1) & 1u, abort_flag, kWaitLimitNs)) {
           ok = false;
           break;
@@ -379,20 +439,20 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           const uint32_t b_base = smem_u32(sB + s * kBBytes);
           const uint32_t t_sf = tmem + kSfSlotCol + slot * kSfSlotCols;
           for (int k = 0; k < nmma; ++k)
-            tc_mma(t_acc, operand_desc(a_base + 32 * k), operand_desc(b_base + 32 * k), idesc,
-                   t_sf + 4 * k, t_sf + 16 + 8 * k, (kt > 0 || k > 0) ? 1u : 0u);
-          tc_commit(smem_u32(&empty[s]));
-          tc_commit(smem_u32(&sf_empty[slot]));
+            tc_mma_pair(t_acc, operand_desc(a_base + 32 * k), operand_desc(b_base + 32 * k), idesc,
+                        t_sf + 4 * k, t_sf + 16 + 8 * k, (kt > 0 || k > 0) ? 1u : 0u);
+          tc_commit_pair(smem_u32(&empty[s]));
+          tc_commit_pair(smem_u32(&sf_empty[slot]));
         }
-        // signals once this tile's MMAs (and everything before) completed
-        tc_commit(smem_u32(&acc_full[b]));
+        // signals both CTAs once this tile's MMAs (and everything before) completed
+        tc_commit_pair(smem_u32(&acc_full[b]));
       }
       if (!ok) {
         *abort_flag = 1;
         atomicOr(p.err, kDevErrTimeout);
       }
-      // no MMA may still run when the CTA frees its tensor memory (bounded)
-      tc_commit(smem_u32(mma_done));
+      // no MMA may still run when the pair frees its tensor memory (bounded)
+      tc_commit_pair(smem_u32(mma_done));
       mbar_wait(smem_u32(mma_done), 0, nullptr, kWaitLimitNs);
     }
   } else if (warp < kSfWarp0) {
@@ -402,11 +462,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const int half = e >> 2;       // 0 / 1: first / second half of each column range
     const float scale = __fmul_rn(*p.a_alpha, *p.b_alpha);
     uint32_t tile_i = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tile_i) {
+    for (int t = pair; t < num_tiles; t += num_pairs, ++tile_i) {
       const uint32_t b = tile_i & 1u, use = tile_i >> 1;
       int mt, nt;
       tile_coords(t, num_m, num_n, mt, nt);
-      const int m0 = mt * BM, n0 = nt * BN;
+      const int m0 = mt * 2 * BM + (int)rank * BM, n0 = nt * BN;
       if (!mbar_wait(smem_u32(&acc_full[b]), use & 1u, abort_flag, kWaitLimitNs)) {
         atomicOr(p.err, kDevErrTimeout);
         *abort_flag = 1;
@@ -434,11 +494,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       drain(ovl_c0 + half * kOvlPer, kOvlPer);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(ovl_free));
+      if (lane == 0) mbar_arrive_leader(smem_u32(ovl_free), leader);
       drain(rest_c0 + half * kRestPer, kRestPer);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
+      if (lane == 0) mbar_arrive_leader(smem_u32(&acc_empty[b]), leader);
     }
   } else {
     // ------------------------------------------------------------ scale staging
@@ -450,11 +510,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     uint32_t it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+    for (int t = pair; t < num_tiles && ok; t += num_pairs) {
       for (int kt = 0; kt < num_kt; ++kt, ++it) {
         const int s = it % kStages;
         const uint32_t slot = it % kSfSlots;
-        if (!mbar_wait(smem_u32(&full[s]), (it / kStages) & 1u, abort_flag, kWaitLimitNs) ||
+        if (!mbar_wait(smem_u32(&sf_in[s]), (it / kStages) & 1u, abort_flag, kWaitLimitNs) ||
             !mbar_wait(smem_u32(&sf_empty[slot]), ((it / kSfSlots) & 1u) ^ 1u, abort_flag,
                        kWaitLimitNs)) {
           ok = false;
@@ -483,7 +543,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&sf_full[slot]));
+        if (lane == 0) mbar_arrive_leader(smem_u32(&sf_full[slot]), leader);
       }
     }
     if (!ok) {
@@ -493,11 +553,14 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   }
 
   // ---------------------------------------------------------------- teardown
+  // neither CTA frees its tensor memory or shared memory while the pair's
+  // MMAs or the other CTA's arrivals may still touch them
   tc_fence_before();
   __syncthreads();
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                  : "memory");
   }
 }
@@ -536,10 +599,27 @@ bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_
   return r == CUDA_SUCCESS;
 }
 
+cudaLaunchConfig_t pair_config(dim3 grid, cudaStream_t s, cudaLaunchAttribute attr[2]) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kNumThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cfg;
+}
+
 int launch_persistent(const GemmArgs& a, cudaStream_t s) {
   CUtensorMap tmA, tmB;
   if (!make_codes_map(&tmA, a.a_codes, a.M, a.K, BM)) return (int)cudaErrorInvalidValue;
-  if (!make_codes_map(&tmB, a.b_codes, a.N, a.K, BN)) return (int)cudaErrorInvalidValue;
+  if (!make_codes_map(&tmB, a.b_codes, a.N, a.K, BN / 2)) return (int)cudaErrorInvalidValue;
   Params p;
   p.a_sf = a.a_sf;
   p.b_sf = a.b_sf;
@@ -553,25 +633,23 @@ int launch_persistent(const GemmArgs& a, cudaStream_t s) {
   p.out_bf16 = a.out_bf16;
   p.epilogue = a.epilogue;
   p.err = a.err;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
-    if (e != cudaSuccess) return (int)e;
-    attr_set = true;
-  }
-  const int64_t tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
-  const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kNumThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  // resident pairs: one pair per two SMs where the GPU's layout allows
+  static const int max_pairs = [] {
+    if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes) != cudaSuccess)
+      return 0;
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = pair_config(dim3(2), nullptr, attr);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel, &cfg) != cudaSuccess || n < 1)
+      n = num_sms() / 2;
+    return n;
+  }();
+  if (max_pairs < 1) return (int)cudaErrorInvalidConfiguration;
+  const int64_t tiles = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + BN - 1) / BN);
+  const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = pair_config(dim3(2 * pairs), s, attr);
   return (int)cudaLaunchKernelEx(&cfg, gemm_kernel, tmA, tmB, p);
 }
 
