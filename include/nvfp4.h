@@ -31,8 +31,16 @@
  *           + (r%32)*16 + ((r%128)/32)*4 + kb%4,
  *         rows padded to a multiple of 128 and blocks to a multiple of 4;
  *         the quantizers write zeros into the padding.
- *   - Pointers to tensors must be 16-byte aligned; leading dimensions are in
- *     elements and must keep every row 16-byte aligned.
+ *   - Alignment (leading dimensions are in elements; a violation returns
+ *     NVFP4_ERR_ALIGN): a quantizer input read along its contiguous rows
+ *     (block_axis 0, and the 2D quantizer) starts on a 32-byte boundary and
+ *     every row does too (ld * element size a multiple of 32); an input read
+ *     across rows (block_axis 1) needs 16 bytes for both.  Codes buffers are
+ *     16-byte aligned (8 for nvfp4_dequantize), scale buffers and global
+ *     scales 4-byte aligned, dequantized outputs 32-byte aligned with 32-byte
+ *     rows, GEMM operands (codes and scales) and outputs 16-byte aligned with
+ *     16-byte output rows; nvfp4_rht16 takes an element-aligned input and a
+ *     4-byte aligned output.
  */
 #ifndef NVFP4_H_
 #define NVFP4_H_
