@@ -44,10 +44,12 @@ def assert_q_equal(q: nv.QTensor, ref, what=""):
 
 def gemm_tolerance(ref_y, ref_s, out_bf16: bool, gelu: bool = False):
     """|gpu - oracle| <= 1e-3 * sum_k |a_k b_k| (+ half a bf16 ulp of the
-    reference for bf16 outputs; the GELU epilogue's slope is below 1.13)."""
+    reference for bf16 outputs).  With the GELU epilogue: its slope is below
+    1.13, and the hardware tanh (relative error about 2^-11) moves GELU(y) by
+    at most 0.5 |y| 2^-11 <= 2.5e-4 * sum_k |a_k b_k|."""
     tol = 1e-3 * ref_s
     if gelu:
-        tol = 1.13 * tol + 1e-6 * np.abs(ref_y) + 1e-30
+        tol = 1.13 * tol + 2.5e-4 * ref_s + 1e-6 * np.abs(ref_y) + 1e-30
     if out_bf16:
         mag = np.abs(ref_y)
         e = np.floor(np.log2(np.where(mag > 0, mag, 1e-300)))
