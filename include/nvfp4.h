@@ -229,6 +229,29 @@ NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor_desc* descs, int32_t 
                               int32_t out_dtype, int32_t sf_layout,
                               void* stream);
 
+/* Gathering dequantization for a sliding-window KV cache with attention
+ * sinks (explainer, section 3.4, "Multi-shot attention sink": the effective
+ * key/value set is the global sink, the shot-level sink given by START and
+ * LEN, and the window KV[t-W, t), overlapping entries deduplicated;
+ * "Parallel CUDA dequantization kernel").  The same source rows of every
+ * tensor are dequantized, in increasing row order, into contiguous output
+ * rows: one launch for all tensors.
+ *   descs[i]: codes, scales (sf_layout), global_scale, out, rows, cols as in
+ *     nvfp4_dequantize; out has room for the gathered rows (ld = row
+ *     stride in elements).
+ *   row_ranges: HOST array of n_ranges pairs {begin, end}, half-open source
+ *     row ranges (for a [heads * tokens, d] cache: head h's tokens [a, b)
+ *     are rows [h*tokens + a, h*tokens + b)).  The ranges are sorted and
+ *     merged on the host (overlapping or touching ranges joined, empty ones
+ *     dropped); output row o is the o-th row of the union.
+ *   n_ranges <= 1024 (NVFP4_ERR_SHAPE beyond); begin < 0, end < begin or a
+ *   union reaching past any tensor's rows: NVFP4_ERR_SHAPE.  Alignment as
+ *   nvfp4_dequantize.  Bit-exact with nvfp4_dequantize on the same rows. */
+NVFP4_API nvfp4_status nvfp4_dequantize_rows(const nvfp4_tensor_desc* descs, int32_t n,
+                                             const int64_t* row_ranges, int32_t n_ranges,
+                                             int32_t out_dtype, int32_t sf_layout,
+                                             void* stream);
+
 /* ------------------------------------------------------------ GEMM ------ */
 
 /* Block-scaled FP4 GEMM on the 5th-generation tensor cores

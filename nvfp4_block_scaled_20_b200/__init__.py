@@ -15,7 +15,8 @@ from .capi import (NVFP4_BF16, NVFP4_EPI_GELU_TANH, NVFP4_EPI_NONE, NVFP4_F32,  
                    NVFP4_SF_ROWMAJOR, NVFP4_SF_TCGEN05, NVFP4Error)
 
 __all__ = ["QTensor", "quantize_1d", "quantize_2d", "global_scale", "quantize_1d_batched",
-           "dequantize", "gemm", "rht16", "workspace", "device_error", "capi"]
+           "dequantize", "dequantize_rows", "window_row_ranges", "gemm", "rht16", "workspace",
+           "device_error", "capi"]
 
 
 def _torch():
@@ -152,6 +153,49 @@ def dequantize(qs, out_dtype=None, outs=None, stream=None):
     code = NVFP4_BF16 if out_dtype == torch.bfloat16 else NVFP4_F32
     st = capi.nvfp4_dequantize(descs, n, code, qs[0].sf_layout, _stream(stream))
     capi.check("nvfp4_dequantize", st)
+    return outs
+
+
+def merged_rows(row_ranges):
+    """Number of rows in the union of half-open ranges (the output height of
+    dequantize_rows)."""
+    total, end = 0, None
+    for b, e in sorted((int(b), int(e)) for b, e in row_ranges if int(e) > int(b)):
+        if end is None or b > end:
+            total += e - b
+            end = e
+        elif e > end:
+            total += e - end
+            end = e
+    return total
+
+
+def window_row_ranges(heads, tokens, token_ranges):
+    """Row ranges of a [heads * tokens, d] cache for the given token ranges of
+    every head (e.g. global sink, shot sink, recent window)."""
+    return [(h * tokens + a, h * tokens + b) for h in range(heads) for a, b in token_ranges]
+
+
+def dequantize_rows(qs, row_ranges, out_dtype=None, outs=None, stream=None):
+    """One nvfp4_dequantize_rows call: the union of row_ranges of every
+    QTensor, in row order, into contiguous outputs."""
+    import ctypes
+    torch = _torch()
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    n = len(qs)
+    rows_out = merged_rows(row_ranges)
+    if outs is None:
+        outs = [torch.empty((rows_out, q.cols), dtype=out_dtype, device=q.codes.device) for q in qs]
+    descs = (capi.nvfp4_tensor_desc * n)()
+    for i, (q, o) in enumerate(zip(qs, outs)):
+        descs[i] = capi.nvfp4_tensor_desc(None, o.data_ptr(), q.codes.data_ptr(),
+                                          q.scales.data_ptr(), q.alpha.data_ptr(), q.rows, q.cols,
+                                          o.stride(0))
+    flat = (ctypes.c_int64 * (2 * len(row_ranges)))(*[v for r in row_ranges for v in r])
+    code = NVFP4_BF16 if out_dtype == torch.bfloat16 else NVFP4_F32
+    st = capi.nvfp4_dequantize_rows(descs, n, flat, len(row_ranges), code, qs[0].sf_layout,
+                                    _stream(stream))
+    capi.check("nvfp4_dequantize_rows", st)
     return outs
 
 

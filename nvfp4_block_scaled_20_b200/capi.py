@@ -22,7 +22,7 @@ NVFP4_EPI_NONE, NVFP4_EPI_GELU_TANH = 0, 1
 EXPORTED = [
     "nvfp4_workspace_bytes", "nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_global_scale",
     "nvfp4_quantize_1d", "nvfp4_quantize_2d", "nvfp4_quantize_1d_batched",
-    "nvfp4_quantize_1d_batched_noalloc", "nvfp4_dequantize",
+    "nvfp4_quantize_1d_batched_noalloc", "nvfp4_dequantize", "nvfp4_dequantize_rows",
     "nvfp4_gemm", "nvfp4_rht16", "nvfp4_get_device_error", "nvfp4_status_string",
 ]
 
@@ -62,6 +62,8 @@ _SIGS = {
     "nvfp4_quantize_1d_batched": (_I32, [_TD, _I32, _I32, _QP, _V, _SZ, _V]),
     "nvfp4_quantize_1d_batched_noalloc": (_I32, [_TD, _I32, _I32, _QP, _V]),
     "nvfp4_dequantize": (_I32, [_TD, _I32, _I32, _I32, _V]),
+    "nvfp4_dequantize_rows": (_I32, [_TD, _I32, ctypes.POINTER(ctypes.c_int64), _I32, _I32, _I32,
+                                     _V]),
     "nvfp4_gemm": (_I32, [_V, _V, _V, _V, _V, _V, _I64, _I64, _I64, _V, _I32, _I64, _I32, _V,
                           _SZ, _V]),
     "nvfp4_rht16": (_I32, [_V, _I32, _I64, _I64, _I64, _I32, _U32, _V, _V]),
@@ -134,6 +136,11 @@ def nvfp4_quantize_1d_batched_noalloc(descs, n, dtype, qp, stream):
 
 def nvfp4_dequantize(descs, n, out_dtype, sf_layout, stream):
     return _call("nvfp4_dequantize", descs, n, out_dtype, sf_layout, stream)
+
+
+def nvfp4_dequantize_rows(descs, n, row_ranges, n_ranges, out_dtype, sf_layout, stream):
+    return _call("nvfp4_dequantize_rows", descs, n, row_ranges, n_ranges, out_dtype, sf_layout,
+                 stream)
 
 
 def nvfp4_gemm(a_codes, a_sf, a_alpha, b_codes, b_sf, b_alpha, M, N, K, out, out_dtype, ldo,

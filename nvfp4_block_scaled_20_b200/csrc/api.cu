@@ -1,7 +1,10 @@
 // C ABI of the NVFP4 library (declared in include/nvfp4.h): argument
 // validation on the host, workspace carve-up, kernel launches.  Nothing here
 // allocates device memory or synchronizes (except nvfp4_get_device_error).
+#include <algorithm>
 #include <cstring>
+#include <memory>
+#include <vector>
 
 #include "../../include/nvfp4.h"
 #include "kernels.h"
@@ -196,6 +199,62 @@ nvfp4_status nvfp4_dequantize(const nvfp4_tensor_desc* descs, int32_t n, int32_t
     }
     if (b.n == 0) continue;
     cudaError_t e = launch_dequantize(b, S(stream));
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  }
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_dequantize_rows(const nvfp4_tensor_desc* descs, int32_t n,
+                                   const int64_t* row_ranges, int32_t n_ranges,
+                                   int32_t out_dtype, int32_t sf_layout, void* stream) {
+  if (!descs || n < 0 || n_ranges < 0 || (n_ranges > 0 && !row_ranges) || !dtype_ok(out_dtype))
+    return NVFP4_ERR_INVALID_ARG;
+  if (sf_layout != NVFP4_SF_ROWMAJOR && sf_layout != NVFP4_SF_TCGEN05) return NVFP4_ERR_INVALID_ARG;
+  if (n_ranges > kMaxRowRanges) return NVFP4_ERR_SHAPE;
+  // merge: sort by begin, join overlapping and touching ranges, drop empty ones
+  std::vector<std::pair<int64_t, int64_t>> r;
+  for (int32_t i = 0; i < n_ranges; ++i) {
+    const int64_t b = row_ranges[2 * i], e = row_ranges[2 * i + 1];
+    if (b < 0 || e < b) return NVFP4_ERR_SHAPE;
+    if (e > b) r.emplace_back(b, e);
+  }
+  std::sort(r.begin(), r.end());
+  std::vector<std::pair<int64_t, int64_t>> m;
+  for (const auto& x : r) {
+    if (!m.empty() && x.first <= m.back().second) m.back().second = std::max(m.back().second, x.second);
+    else m.push_back(x);
+  }
+  const int64_t last = m.empty() ? 0 : m.back().second;
+  for (int32_t i = 0; i < n; ++i) {
+    const nvfp4_tensor_desc& d = descs[i];
+    if (!d.codes || !d.scales || !d.global_scale || !d.out) return NVFP4_ERR_INVALID_ARG;
+    if (d.rows < 0 || d.cols < 0 || d.cols % 16 || d.ld < d.cols || last > d.rows)
+      return NVFP4_ERR_SHAPE;
+    if ((double)d.rows * (double)d.cols / 16.0 >= 4.0e9) return NVFP4_ERR_SHAPE;
+    if (!aligned(d.codes, 8) || !aligned(d.out, 32) || (d.ld * elem_bytes(out_dtype)) % 32)
+      return NVFP4_ERR_ALIGN;
+  }
+  if (m.empty() || n == 0) return NVFP4_OK;
+  // large (about 24 KB): kept off the host stack
+  std::unique_ptr<DQGather> g(new DQGather);
+  std::memset(g.get(), 0, sizeof(DQGather));
+  g->n_ranges = (int32_t)m.size();
+  g->prefix[0] = 0;
+  for (size_t i = 0; i < m.size(); ++i) {
+    g->begin[i] = m[i].first;
+    g->prefix[i + 1] = g->prefix[i] + (m[i].second - m[i].first);
+  }
+  g->b.out_bf16 = out_dtype == NVFP4_BF16;
+  g->b.sf_layout = sf_layout;
+  for (int32_t base = 0; base < n; base += kMaxBatch) {
+    g->b.n = 0;
+    for (int32_t i = base; i < n && i < base + kMaxBatch; ++i) {
+      const nvfp4_tensor_desc& d = descs[i];
+      if (d.cols == 0) continue;
+      g->b.t[g->b.n++] = DQTensor{d.codes, d.scales, d.global_scale, d.out, d.rows, d.cols, d.ld};
+    }
+    if (g->b.n == 0) continue;
+    cudaError_t e = launch_dequantize_rows(*g, S(stream));
     if (e != cudaSuccess) return NVFP4_ERR_CUDA;
   }
   return NVFP4_OK;

@@ -53,6 +53,17 @@ struct DQBatch {
   int32_t sf_layout;
 };
 
+// Row-gather dequantization: the same source rows of every tensor, given as
+// disjoint sorted ranges [begin[i], begin[i] + len_i); output row o comes
+// from range i where prefix[i] <= o < prefix[i + 1].
+constexpr int kMaxRowRanges = 1024;
+struct DQGather {
+  DQBatch b;
+  int32_t n_ranges;
+  int64_t begin[kMaxRowRanges];
+  int64_t prefix[kMaxRowRanges + 1];
+};
+
 struct GemmArgs {
   const uint8_t* a_codes;
   const uint8_t* a_sf;
@@ -77,6 +88,7 @@ int num_sms();
 // kernel and a finalize kernel when amax_only is set.
 cudaError_t launch_quantize(const QBatch& b, cudaStream_t s);
 cudaError_t launch_dequantize(const DQBatch& b, cudaStream_t s);
+cudaError_t launch_dequantize_rows(const DQGather& g, cudaStream_t s);
 cudaError_t launch_rht16(const void* x, int bf16, int64_t rows, int64_t cols, int64_t ld,
                          int block_axis, uint32_t mask, float* out, cudaStream_t s);
 // Returns 0 on success, a cudaError_t value otherwise; sets *unsupported for

@@ -584,6 +584,42 @@ uint64_t max_units(const QBatch& b, int mode) {
 // Dequantization, one 16-block per thread step, all tensors of a batch in
 // one launch (tensor = blockIdx.y).
 template <bool BF16>
+__device__ __forceinline__ void dequant_block(const DQTensor& q, int64_t r, uint32_t kb,
+                                              uint32_t kbpr, int sf_layout, uint64_t aa,
+                                              int64_t out_row) {
+  const uint2 c = __ldg(reinterpret_cast<const uint2*>(q.codes + r * (q.cols >> 1) + (int64_t)kb * 8));
+  const float d = e4m3_to_f32(__ldg(q.scales + sf_offset(r, kb, kbpr, sf_layout)));
+  const uint64_t dd = pack2(d, d);
+  float o[16];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t byte = ((k < 4 ? c.x : c.y) >> (8 * (k & 3))) & 0xFFu;
+    const uint64_t vd = mul2(e2m1x2_to_f32x2(byte), dd);  // exact
+    unpack2(mul2(vd, aa), o[2 * k], o[2 * k + 1]);
+  }
+  if (BF16) {
+    uint32_t w[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(o[2 * k], o[2 * k + 1]);
+      w[k] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(q.out) + out_row * q.ldo + (int64_t)kb * 16;
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst), "r"(w[0]),
+                 "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+  } else {
+    float* dst = static_cast<float*>(q.out) + out_row * q.ldo + (int64_t)kb * 16;
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst + 8 * h),
+                   "f"(o[8 * h]), "f"(o[8 * h + 1]), "f"(o[8 * h + 2]), "f"(o[8 * h + 3]),
+                   "f"(o[8 * h + 4]), "f"(o[8 * h + 5]), "f"(o[8 * h + 6]), "f"(o[8 * h + 7])
+                   : "memory");
+  }
+}
+
+template <bool BF16>
 __global__ void __launch_bounds__(kThreads) dequant_kernel(const __grid_constant__ DQBatch p) {
   const DQTensor& q = p.t[blockIdx.y];
   const float alpha = *q.gs;
@@ -593,37 +629,32 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(const __grid_constant
   for (uint64_t u = (uint64_t)blockIdx.x * kThreads + threadIdx.x; u < nblk;
        u += (uint64_t)gridDim.x * kThreads) {
     const uint32_t r = (uint32_t)u / kbpr, kb = (uint32_t)u - r * kbpr;
-    const uint2 c = __ldg(reinterpret_cast<const uint2*>(q.codes + (int64_t)r * (q.cols >> 1) +
-                                                         (int64_t)kb * 8));
-    const float d = e4m3_to_f32(__ldg(q.scales + sf_offset(r, kb, kbpr, p.sf_layout)));
-    const uint64_t dd = pack2(d, d);
-    float o[16];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t byte = ((k < 4 ? c.x : c.y) >> (8 * (k & 3))) & 0xFFu;
-      const uint64_t vd = mul2(e2m1x2_to_f32x2(byte), dd);  // exact
-      unpack2(mul2(vd, aa), o[2 * k], o[2 * k + 1]);
+    dequant_block<BF16>(q, r, kb, kbpr, p.sf_layout, aa, r);
+  }
+}
+
+// Row-gather dequantization: output row o of every tensor is source row
+// begin[i] + (o - prefix[i]) for the range i holding o (binary search over
+// the merged ranges).
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads) dequant_rows_kernel(const __grid_constant__ DQGather g) {
+  const DQTensor& q = g.b.t[blockIdx.y];
+  const float alpha = *q.gs;
+  const uint64_t aa = pack2(alpha, alpha);
+  const uint32_t kbpr = (uint32_t)(q.cols >> 4);
+  const int64_t rows_out = g.prefix[g.n_ranges];
+  const uint64_t nblk = (uint64_t)rows_out * kbpr;
+  for (uint64_t u = (uint64_t)blockIdx.x * kThreads + threadIdx.x; u < nblk;
+       u += (uint64_t)gridDim.x * kThreads) {
+    const int64_t o = (int64_t)(u / kbpr);
+    const uint32_t kb = (uint32_t)(u - (uint64_t)o * kbpr);
+    int lo = 0, hi = g.n_ranges - 1;  // last range with prefix <= o
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (g.prefix[mid] <= o) lo = mid;
+      else hi = mid - 1;
     }
-    if (BF16) {
-      uint32_t w[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(o[2 * k], o[2 * k + 1]);
-        w[k] = *reinterpret_cast<uint32_t*>(&h);
-      }
-      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(q.out) + (int64_t)r * q.ldo + (int64_t)kb * 16;
-      asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst), "r"(w[0]),
-                   "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
-                   : "memory");
-    } else {
-      float* dst = static_cast<float*>(q.out) + (int64_t)r * q.ldo + (int64_t)kb * 16;
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-        asm volatile("st.global.v8.f32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst + 8 * h),
-                     "f"(o[8 * h]), "f"(o[8 * h + 1]), "f"(o[8 * h + 2]), "f"(o[8 * h + 3]),
-                     "f"(o[8 * h + 4]), "f"(o[8 * h + 5]), "f"(o[8 * h + 6]), "f"(o[8 * h + 7])
-                     : "memory");
-    }
+    dequant_block<BF16>(q, g.begin[lo] + (o - g.prefix[lo]), kb, kbpr, g.b.sf_layout, aa, o);
   }
 }
 
@@ -748,6 +779,21 @@ cudaError_t launch_dequantize(const DQBatch& b, cudaStream_t s) {
     dequant_kernel<true><<<grid, kThreads, 0, s>>>(b);
   else
     dequant_kernel<false><<<grid, kThreads, 0, s>>>(b);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize_rows(const DQGather& g, cudaStream_t s) {
+  const uint64_t m = (uint64_t)g.prefix[g.n_ranges] * (uint64_t)(g.b.t[0].cols / 16);
+  uint64_t mx = m;
+  for (int i = 1; i < g.b.n; ++i) {
+    const uint64_t u = (uint64_t)g.prefix[g.n_ranges] * (uint64_t)(g.b.t[i].cols / 16);
+    mx = u > mx ? u : mx;
+  }
+  dim3 grid(grid_for(mx, g.b.n), g.b.n);
+  if (g.b.out_bf16)
+    dequant_rows_kernel<true><<<grid, kThreads, 0, s>>>(g);
+  else
+    dequant_rows_kernel<false><<<grid, kThreads, 0, s>>>(g);
   return cudaGetLastError();
 }
 

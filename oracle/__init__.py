@@ -92,6 +92,8 @@ def lib():
                                ctypes.c_float, _i32, _i64, _i64, _i64, _F64P, _F64P]
         L.orc_gelu_tanh.restype = ctypes.c_double
         L.orc_gelu_tanh.argtypes = [ctypes.c_double]
+        L.orc_transpose_2d.restype = _i32
+        L.orc_transpose_2d.argtypes = [_U8P, _U8P, _i64, _i64, _i32, _U8P, _U8P, _i32]
         _lib = L
     return _lib
 
@@ -214,6 +216,21 @@ def dequantize(codes, scales, alpha: float, rows: int, cols: int,
     lib().orc_dequantize(_p(codes, _U8P), _p(scales, _U8P), float(alpha), rows, cols,
                          sf_layout, _p(out32, _F32P), _p(out16, _U16P))
     return out32, out16
+
+
+def transpose_2d(codes, scales, rows: int, cols: int, sf_layout_in: int = SF_ROWMAJOR,
+                 sf_layout_out: int = SF_ROWMAJOR):
+    """The encoding of W^T read off a 2D (16x16-tile) encoding of W [rows, cols]:
+    returns (codes [cols, rows/2], scales for cols rows x rows/16 blocks)."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    out_codes = np.zeros((cols, rows // 2), dtype=np.uint8)
+    out_scales = np.zeros(sf_bytes(cols, rows // 16, sf_layout_out), dtype=np.uint8)
+    rc = lib().orc_transpose_2d(_p(codes, _U8P), _p(scales, _U8P), rows, cols, sf_layout_in,
+                                _p(out_codes, _U8P), _p(out_scales, _U8P), sf_layout_out)
+    if rc != 0:
+        raise ValueError("bad shape for transpose_2d")
+    return out_codes, out_scales
 
 
 # ---------------------------------------------------------------- GEMM

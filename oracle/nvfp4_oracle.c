@@ -441,6 +441,38 @@ void orc_dequantize(const uint8_t* codes, const uint8_t* scales, float alpha,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Transpose of a 2D (16x16-tile) encoding, for the data-gradient GEMM        */
+/* ------------------------------------------------------------------------ */
+
+/* The data-gradient GEMM dA = dO . W contracts W along its output dimension
+ * ("The three GEMMs of backpropagation in NVFP4": DGRAD takes W in NVFP4),
+ * so it needs W^T blocked along W's rows.  With one scale per 16x16 tile
+ * ("Quantization rule for a tensor block", 2D blocks for weights) the
+ * encoding of W already holds W^T's blocks: element (c, r) of the output is
+ * element (r, c) of the input, and output block (c, b) -- 16 elements along
+ * W's rows 16b .. 16b+15 -- has the scale of the tile (b, c/16), read from
+ * input row 16b.  rows and cols are multiples of 16.  Returns 0, or -1 on a
+ * bad shape. */
+int orc_transpose_2d(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                     int sf_layout_in, uint8_t* out_codes, uint8_t* out_scales,
+                     int sf_layout_out) {
+  if (rows < 0 || cols < 0 || rows % 16 || cols % 16) return -1;
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t c = 0; c < cols; ++c) {
+      uint8_t byte = codes[r * (cols / 2) + c / 2];
+      uint8_t q = (uint8_t)((c & 1) ? (byte >> 4) : (byte & 15));
+      put_code(out_codes, rows / 2, c, r, q);
+    }
+  }
+  int64_t out_kb = rows / 16, in_kb = cols / 16;
+  for (int64_t c = 0; c < cols; ++c)
+    for (int64_t b = 0; b < out_kb; ++b)
+      out_scales[orc_sf_offset(c, b, out_kb, sf_layout_out)] =
+          scales[orc_sf_offset(16 * b, c / 16, in_kb, sf_layout_in)];
+  return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* GEMM reference on the encodings: Y[m,n] = sum_k a^_mk * b^_nk (fp64)       */
 /* ------------------------------------------------------------------------ */
 

@@ -119,3 +119,52 @@ def test_rht_validation(lib):
     assert capi.nvfp4_rht16(A, 1, 64, 100, 100, 0, 0, A, None) == 2
     assert capi.nvfp4_rht16(A, 1, 60, 64, 64, 1, 0, A, None) == 2
     assert capi.nvfp4_rht16(A, 1, 64, 64, 64, 2, 0, A, None) == 1
+
+
+def _ranges(pairs):
+    flat = [v for p in pairs for v in p]
+    return (ctypes.c_int64 * max(1, len(flat)))(*flat)
+
+
+def test_dequantize_rows_validation(lib):
+    e = (capi.nvfp4_tensor_desc * 1)()
+    e[0] = capi.nvfp4_tensor_desc(None, A, A, A, A, 64, 128, 128)
+    r = _ranges([(0, 8), (32, 40)])
+    assert capi.nvfp4_dequantize_rows(e, 1, None, 2, 1, 0, None) == 1   # ranges missing
+    assert capi.nvfp4_dequantize_rows(e, 1, _ranges([(-1, 4)]), 1, 1, 0, None) == 2
+    assert capi.nvfp4_dequantize_rows(e, 1, _ranges([(9, 4)]), 1, 1, 0, None) == 2
+    assert capi.nvfp4_dequantize_rows(e, 1, _ranges([(60, 65)]), 1, 1, 0, None) == 2  # past rows
+    assert capi.nvfp4_dequantize_rows(e, 1, r, 1025, 1, 0, None) == 2   # more than 1024 ranges
+    assert capi.nvfp4_dequantize_rows(e, 1, r, 2, 7, 0, None) == 1      # unknown dtype
+    assert capi.nvfp4_dequantize_rows(e, 1, r, 2, 1, 3, None) == 1      # unknown layout
+    e[0] = capi.nvfp4_tensor_desc(None, A, A, A, A, 64, 120, 128)
+    assert capi.nvfp4_dequantize_rows(e, 1, r, 2, 1, 0, None) == 2      # cols % 16
+    # empty union or no tensors: nothing to do, nothing launched
+    assert capi.nvfp4_dequantize_rows(e, 0, r, 2, 1, 0, None) == 0
+    e[0] = capi.nvfp4_tensor_desc(None, A, A, A, A, 64, 128, 128)
+    assert capi.nvfp4_dequantize_rows(e, 1, _ranges([(5, 5)]), 1, 1, 0, None) == 0
+
+
+def test_window_rows_helpers_match_a_set_union():
+    """The binding's output height and head-wise ranges against a brute-force
+    set of row indices."""
+    import random
+    import nvfp4_block_scaled_20_b200 as nv
+    rnd = random.Random(7)
+    for _ in range(200):
+        rr = []
+        for _ in range(rnd.randrange(0, 6)):
+            b = rnd.randrange(0, 50)
+            rr.append((b, b + rnd.randrange(0, 12)))
+        want = set()
+        for b, e in rr:
+            want.update(range(b, e))
+        assert nv.merged_rows(rr) == len(want)
+    heads, tokens = 3, 40
+    tr = [(0, 4), (10, 14), (30, 40), (12, 20)]
+    rows = nv.window_row_ranges(heads, tokens, tr)
+    want = {h * tokens + t for h in range(heads) for a, b in tr for t in range(a, b)}
+    got = set()
+    for b, e in rows:
+        got.update(range(b, e))
+    assert got == want and nv.merged_rows(rows) == len(want)

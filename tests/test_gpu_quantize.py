@@ -217,3 +217,29 @@ def test_dequant_tcgen05_layout():
     ref = oracle.quantize_2d(to_oracle(w), sf_layout=oracle.SF_TCGEN05)
     d32, _ = oracle.dequantize(ref[0], ref[1], ref[2], 160, 512, oracle.SF_TCGEN05)
     assert np.array_equal(out.view(np.uint32), d32.view(np.uint32))
+
+
+@pytest.mark.parametrize("layout", [nv.NVFP4_SF_ROWMAJOR, nv.NVFP4_SF_TCGEN05])
+def test_window_gather_dequant(layout):
+    """Global sink, shot sink (START, LEN) and recent window of every head,
+    overlapping and touching ranges included, against the oracle's dequant
+    of the union of those rows (in row order), bit for bit."""
+    heads, tokens = 6, 300
+    ts = [synth.kv_tensor(3, l, w, heads=heads, tokens=tokens) for l in range(2) for w in range(2)]
+    qs = nv.quantize_1d_batched([t.to(DEV) for t in ts], sf_layout=layout)
+    token_ranges = [(0, 8), (100, 108), (104, 112), (112, 120), (250, 300), (299, 300), (7, 7)]
+    ranges = nv.window_row_ranges(heads, tokens, token_ranges)
+    rows = sorted({r for b, e in ranges for r in range(b, e)})
+    for dt in (torch.bfloat16, torch.float32):
+        outs = nv.dequantize_rows(qs, ranges, out_dtype=dt)
+        for t, q, o in zip(ts, qs, outs):
+            assert o.shape[0] == len(rows)
+            ref = oracle.quantize_1d(to_oracle(t), sf_layout=layout)
+            d32, d16 = oracle.dequantize(ref[0], ref[1], ref[2], t.shape[0], t.shape[1], layout)
+            if dt == torch.bfloat16:
+                got = o.cpu().view(torch.int16).numpy().view(np.uint16)
+                want = d16[rows]
+            else:
+                got = o.cpu().numpy().view(np.uint32)
+                want = d32[rows].view(np.uint32)
+            assert np.array_equal(got, want), mismatch_report(got, want, "gather dequant")
