@@ -578,7 +578,23 @@ def measure_rows(nv, synth, torch, dev, stream, timed, pk, reps):
 
     ffn = tc(ffn_step, 4.0 * Mf * Hd * D)
     ffn["note"] = "quantize X, up GEMM + GELU, quantize H, down GEMM (weights pre-quantized)"
-    del x, wu, wd, qx, qu, qd, qh, h, y
+
+    # data gradient of the down projection: dX [8192, 14336] = dY [8192, 3072] . W_dn,
+    # W_dn's 2D encoding transposed (no re-quantization)
+    dyf = synth.activation(2, 7, Mf, D, n_out=0, std=1e-3, device=dev)
+    torch.cuda.synchronize(dev)
+    qdy, qdt = q(Mf, D), q(Hd, D)
+    qdt.alpha = qd.alpha
+    dx = torch.empty((Mf, Hd), dtype=torch.bfloat16, device=dev)
+    nv.quantize_1d(dyf, out=qdy, ws=ws, stream=stream)
+    out["next1_dgrad"] = {
+        "transpose_2d_W_dn_3072x14336": bw(
+            lambda: nv.transpose_2d(qd, out=qdt, stream=stream), 2 * (0.5 + 1.0 / 16) * Hd * D,
+            "codes and tile scales read once and written once"),
+        "dgrad_gemm_8192x14336x3072": tc(lambda: nv.gemm(qdy, qdt, out=dx, ws=ws, stream=stream),
+                                         2.0 * Mf * Hd * D),
+    }
+    del x, wu, wd, qx, qu, qd, qh, h, y, dyf, qdy, qdt, dx
 
     # ---------------- weight gradient
     dy, xw, mask = synth.wgrad(dev)
@@ -623,6 +639,17 @@ def measure_rows(nv, synth, torch, dev, stream, timed, pk, reps):
     out["a7_kv_dequant_batched"] = bw(
         lambda: nv.dequantize(kq, outs=kout, stream=stream), (qout + 2) * ne_kv,
         "60 tensors, one launch")
+    # sliding window with sinks: frames of 1560 tokens (32760 = 21 frames);
+    # global sink frames [0, 3), shot sink frames [6, 9), window frames [12, 21)
+    fr = 1560
+    token_ranges = [(0, 3 * fr), (6 * fr, 9 * fr), (12 * fr, 21 * fr)]
+    ranges = nv.window_row_ranges(24, R // 24, token_ranges)
+    rows_w = nv.merged_rows(ranges)
+    wout = [o[:rows_w] for o in kout]
+    out["next2_window_gather_dequant"] = bw(
+        lambda: nv.dequantize_rows(kq, ranges, outs=wout, stream=stream),
+        (qout + 2) * len(kv) * rows_w * C,
+        "60 tensors, 24 heads x (3 + 3 + 9 of 21 frames), one launch")
     del kv, kq, kout
     assert nv.device_error(ws, stream) == 0 and nv.device_error(ws_kv, stream) == 0
     torch.cuda.empty_cache()

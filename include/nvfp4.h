@@ -229,6 +229,25 @@ NVFP4_API nvfp4_status nvfp4_dequantize(const nvfp4_tensor_desc* descs, int32_t 
                               int32_t out_dtype, int32_t sf_layout,
                               void* stream);
 
+/* Transpose of a 2D (16x16-tile) encoding (explainer, section 3.4, "The
+ * three GEMMs of backpropagation in NVFP4": the data-gradient GEMM
+ * dA = dO . W takes the weight in NVFP4, contracted along W's rows; with one
+ * scale per 16x16 tile the encoding of W holds W^T's blocks, so the codes are
+ * transposed and no element is re-quantized).
+ *   codes [rows, cols/2], scales (sf_layout_in): an encoding written by
+ *     nvfp4_quantize_2d of a [rows, cols] matrix (every row of a tile holds
+ *     the tile's scale; the output takes each tile's first row).
+ *   out_codes [cols, rows/2], out_scales (sf_layout_out, cols rows x
+ *     rows/16 blocks; nvfp4_scales_bytes(cols, rows, layout) bytes): the
+ *     encoding of the transpose, ready as the B operand of nvfp4_gemm.  The
+ *     global scale is unchanged (the caller reuses it).
+ *   rows, cols multiples of 16 (NVFP4_ERR_SHAPE); codes buffers 8-byte
+ *   aligned.  Bit-exact with the transposed oracle encoding. */
+NVFP4_API nvfp4_status nvfp4_transpose_2d(const uint8_t* codes, const uint8_t* scales,
+                                          int32_t sf_layout_in, int64_t rows, int64_t cols,
+                                          uint8_t* out_codes, uint8_t* out_scales,
+                                          int32_t sf_layout_out, void* stream);
+
 /* Gathering dequantization for a sliding-window KV cache with attention
  * sinks (explainer, section 3.4, "Multi-shot attention sink": the effective
  * key/value set is the global sink, the shot-level sink given by START and

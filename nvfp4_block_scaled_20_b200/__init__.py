@@ -15,7 +15,7 @@ from .capi import (NVFP4_BF16, NVFP4_EPI_GELU_TANH, NVFP4_EPI_NONE, NVFP4_F32,  
                    NVFP4_SF_ROWMAJOR, NVFP4_SF_TCGEN05, NVFP4Error)
 
 __all__ = ["QTensor", "quantize_1d", "quantize_2d", "global_scale", "quantize_1d_batched",
-           "dequantize", "dequantize_rows", "window_row_ranges", "gemm", "rht16", "workspace",
+           "dequantize", "dequantize_rows", "window_row_ranges", "transpose_2d", "gemm", "rht16", "workspace",
            "device_error", "capi"]
 
 
@@ -197,6 +197,20 @@ def dequantize_rows(qs, row_ranges, out_dtype=None, outs=None, stream=None):
                                     _stream(stream))
     capi.check("nvfp4_dequantize_rows", st)
     return outs
+
+
+def transpose_2d(q: QTensor, sf_layout=None, out=None, stream=None):
+    """The encoding of the transpose of a 2D-quantized matrix (codes
+    transposed, tile scales carried over, global scale shared)."""
+    sf_layout = q.sf_layout if sf_layout is None else sf_layout
+    if out is None:
+        codes, scales, _ = _alloc_q(q.cols, q.rows, sf_layout, q.codes.device)
+        out = QTensor(codes, scales, q.alpha, q.cols, q.rows, sf_layout)
+    st = capi.nvfp4_transpose_2d(q.codes.data_ptr(), q.scales.data_ptr(), q.sf_layout, q.rows,
+                                 q.cols, out.codes.data_ptr(), out.scales.data_ptr(), sf_layout,
+                                 _stream(stream))
+    capi.check("nvfp4_transpose_2d", st)
+    return out
 
 
 def gemm(a: QTensor, b: QTensor, out_dtype=None, epilogue=NVFP4_EPI_NONE, out=None, ws=None,

@@ -23,6 +23,7 @@ EXPORTED = [
     "nvfp4_workspace_bytes", "nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_global_scale",
     "nvfp4_quantize_1d", "nvfp4_quantize_2d", "nvfp4_quantize_1d_batched",
     "nvfp4_quantize_1d_batched_noalloc", "nvfp4_dequantize", "nvfp4_dequantize_rows",
+    "nvfp4_transpose_2d",
     "nvfp4_gemm", "nvfp4_rht16", "nvfp4_get_device_error", "nvfp4_status_string",
 ]
 
@@ -62,6 +63,7 @@ _SIGS = {
     "nvfp4_quantize_1d_batched": (_I32, [_TD, _I32, _I32, _QP, _V, _SZ, _V]),
     "nvfp4_quantize_1d_batched_noalloc": (_I32, [_TD, _I32, _I32, _QP, _V]),
     "nvfp4_dequantize": (_I32, [_TD, _I32, _I32, _I32, _V]),
+    "nvfp4_transpose_2d": (_I32, [_V, _V, _I32, _I64, _I64, _V, _V, _I32, _V]),
     "nvfp4_dequantize_rows": (_I32, [_TD, _I32, ctypes.POINTER(ctypes.c_int64), _I32, _I32, _I32,
                                      _V]),
     "nvfp4_gemm": (_I32, [_V, _V, _V, _V, _V, _V, _I64, _I64, _I64, _V, _I32, _I64, _I32, _V,
@@ -136,6 +138,12 @@ def nvfp4_quantize_1d_batched_noalloc(descs, n, dtype, qp, stream):
 
 def nvfp4_dequantize(descs, n, out_dtype, sf_layout, stream):
     return _call("nvfp4_dequantize", descs, n, out_dtype, sf_layout, stream)
+
+
+def nvfp4_transpose_2d(codes, scales, sf_layout_in, rows, cols, out_codes, out_scales,
+                       sf_layout_out, stream):
+    return _call("nvfp4_transpose_2d", codes, scales, sf_layout_in, rows, cols, out_codes,
+                 out_scales, sf_layout_out, stream)
 
 
 def nvfp4_dequantize_rows(descs, n, row_ranges, n_ranges, out_dtype, sf_layout, stream):

@@ -260,6 +260,21 @@ nvfp4_status nvfp4_dequantize_rows(const nvfp4_tensor_desc* descs, int32_t n,
   return NVFP4_OK;
 }
 
+nvfp4_status nvfp4_transpose_2d(const uint8_t* codes, const uint8_t* scales,
+                                int32_t sf_layout_in, int64_t rows, int64_t cols,
+                                uint8_t* out_codes, uint8_t* out_scales, int32_t sf_layout_out,
+                                void* stream) {
+  auto layout_ok = [](int32_t l) { return l == NVFP4_SF_ROWMAJOR || l == NVFP4_SF_TCGEN05; };
+  if (!layout_ok(sf_layout_in) || !layout_ok(sf_layout_out)) return NVFP4_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0 || rows % 16 || cols % 16) return NVFP4_ERR_SHAPE;
+  if ((double)rows * (double)cols / 16.0 >= 4.0e9) return NVFP4_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return NVFP4_OK;
+  if (!codes || !scales || !out_codes || !out_scales) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(codes, 8) || !aligned(out_codes, 8)) return NVFP4_ERR_ALIGN;
+  return cuda_status(launch_transpose_2d(codes, scales, sf_layout_in, rows, cols, out_codes,
+                                         out_scales, sf_layout_out, S(stream)));
+}
+
 nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_alpha,
                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_alpha,
                         int64_t M, int64_t N, int64_t K, void* out, int32_t out_dtype, int64_t ldo,

@@ -89,6 +89,9 @@ int num_sms();
 cudaError_t launch_quantize(const QBatch& b, cudaStream_t s);
 cudaError_t launch_dequantize(const DQBatch& b, cudaStream_t s);
 cudaError_t launch_dequantize_rows(const DQGather& g, cudaStream_t s);
+cudaError_t launch_transpose_2d(const uint8_t* codes, const uint8_t* scales, int sf_in,
+                                int64_t rows, int64_t cols, uint8_t* out_codes,
+                                uint8_t* out_scales, int sf_out, cudaStream_t s);
 cudaError_t launch_rht16(const void* x, int bf16, int64_t rows, int64_t cols, int64_t ld,
                          int block_axis, uint32_t mask, float* out, cudaStream_t s);
 // Returns 0 on success, a cudaError_t value otherwise; sets *unsupported for

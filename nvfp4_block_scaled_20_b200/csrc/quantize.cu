@@ -659,6 +659,48 @@ __global__ void __launch_bounds__(kThreads) dequant_rows_kernel(const __grid_con
 }
 
 // ------------------------------------------------------------------------
+// Transpose of a 2D (16x16-tile) encoding: the data-gradient GEMM's weight
+// operand.  A CTA moves 64 x 64 codes through shared memory (one byte per
+// code; rows padded to 68 bytes so the column reads hit 32 different banks)
+// and writes each output block's scale from its tile: output (c, b) takes
+// input (16 b, c / 16).  rows and cols are multiples of 16.
+__global__ void __launch_bounds__(kThreads)
+    transpose_2d_kernel(const uint8_t* codes, const uint8_t* scales, int sf_in, int64_t rows,
+                        int64_t cols, uint8_t* out_codes, uint8_t* out_scales, int sf_out) {
+  __shared__ uint8_t t[64][68];
+  const int64_t tiles_c = (cols + 63) / 64;
+  const int64_t ntiles = ((rows + 63) / 64) * tiles_c;
+  const int lr = threadIdx.x >> 2, part = threadIdx.x & 3;
+  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int64_t r0 = (tile / tiles_c) * 64, c0 = (tile % tiles_c) * 64;
+    {  // thread: row r0 + lr, codes c0 + 16 part .. + 15
+      const int64_t r = r0 + lr, c = c0 + 16 * part;
+      uint2 w = make_uint2(0u, 0u);
+      if (r < rows && c < cols) w = __ldg(reinterpret_cast<const uint2*>(codes + r * (cols >> 1) + (c >> 1)));
+#pragma unroll
+      for (int i = 0; i < 16; ++i) t[lr][16 * part + i] = (uint8_t)(((i < 8 ? w.x : w.y) >> (4 * (i & 7))) & 0xFu);
+    }
+    __syncthreads();
+    {  // thread: output row c0 + lr (input column), codes along rows r0 + 16 part .. + 15
+      const int64_t c = c0 + lr, r = r0 + 16 * part;
+      if (c < cols && r < rows) {
+        uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          lo |= (uint32_t)t[16 * part + i][lr] << (4 * i);
+          hi |= (uint32_t)t[16 * part + 8 + i][lr] << (4 * i);
+        }
+        *reinterpret_cast<uint2*>(out_codes + c * (rows >> 1) + (r >> 1)) = make_uint2(lo, hi);
+        out_scales[sf_offset(c, r >> 4, rows >> 4, sf_out)] =
+            __ldg(scales + sf_offset(r, c >> 4, cols >> 4, sf_in));
+      }
+    }
+    __syncthreads();
+  }
+  if (sf_out == 1) zero_sf_padding(out_scales, cols, rows >> 4);
+}
+
+// ------------------------------------------------------------------------
 // Standalone RHT16 (parity tool for the fused transform): fp32 output.
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
@@ -794,6 +836,17 @@ cudaError_t launch_dequantize_rows(const DQGather& g, cudaStream_t s) {
     dequant_rows_kernel<true><<<grid, kThreads, 0, s>>>(g);
   else
     dequant_rows_kernel<false><<<grid, kThreads, 0, s>>>(g);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_2d(const uint8_t* codes, const uint8_t* scales, int sf_in,
+                                int64_t rows, int64_t cols, uint8_t* out_codes,
+                                uint8_t* out_scales, int sf_out, cudaStream_t s) {
+  const uint64_t tiles = (uint64_t)((rows + 63) / 64) * (uint64_t)((cols + 63) / 64);
+  const uint64_t cap = (uint64_t)num_sms() * 8;
+  const int grid = (int)(tiles < cap ? (tiles < 1 ? 1 : tiles) : cap);
+  transpose_2d_kernel<<<grid, kThreads, 0, s>>>(codes, scales, sf_in, rows, cols, out_codes,
+                                               out_scales, sf_out);
   return cudaGetLastError();
 }
 

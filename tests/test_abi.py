@@ -168,3 +168,12 @@ def test_window_rows_helpers_match_a_set_union():
     for b, e in rows:
         got.update(range(b, e))
     assert got == want and nv.merged_rows(rows) == len(want)
+
+
+def test_transpose_2d_validation(lib):
+    assert capi.nvfp4_transpose_2d(A, A, 0, 64, 120, A, A, 0, None) == 2   # cols % 16
+    assert capi.nvfp4_transpose_2d(A, A, 0, 60, 128, A, A, 0, None) == 2   # rows % 16
+    assert capi.nvfp4_transpose_2d(A, A, 2, 64, 128, A, A, 0, None) == 1   # layout
+    assert capi.nvfp4_transpose_2d(None, A, 0, 64, 128, A, A, 0, None) == 1
+    assert capi.nvfp4_transpose_2d(A + 4, A, 0, 64, 128, A, A, 0, None) == 3  # codes alignment
+    assert capi.nvfp4_transpose_2d(None, None, 0, 0, 128, None, None, 0, None) == 0  # empty

@@ -262,3 +262,37 @@ def test_wgrad_full():
     yr, sr = oracle.gemm((dyr[0], dyr[1], a_dy, oracle.SF_ROWMAJOR),
                          (xr[0], xr[1], a_x, oracle.SF_ROWMAJOR), len(mi), len(ni), T)
     check_gemm(grid(dw, mi, ni), yr, sr, False, what="dW")
+
+
+# ------------------------------------------------------------------ DGRAD
+def test_dgrad_down_projection_full():
+    """dX [8192, 14336] = dY [8192, 3072] . W_dn [3072, 14336] on W_dn's 2D
+    encoding transposed on the GPU: transposed codes and scales whole, the
+    GEMM on a sampled grid."""
+    _, _, wd = synth.ffn_pair(DEV)
+    dy = synth.activation(2, 7, 8192, 3072, n_out=0, std=1e-3, device=DEV)
+    ws = nv.workspace(1)
+    qd = nv.quantize_2d(wd, ws=ws)
+    qt = nv.transpose_2d(qd)
+    qy = nv.quantize_1d(dy, ws=ws)
+    dx = nv.gemm(qy, qt, out_dtype=torch.bfloat16, ws=ws)
+    torch.cuda.synchronize()
+    assert nv.device_error(ws) == 0
+    D, Hd = wd.shape
+    dref = oracle.quantize_2d(host_f32(wd), sf_layout=oracle.SF_TCGEN05)
+    tc, ts = oracle.transpose_2d(dref[0], dref[1], D, Hd, oracle.SF_TCGEN05, oracle.SF_TCGEN05)
+    msg = (mismatch_report(qt.codes.cpu().numpy(), tc, "W_dn^T codes")
+           + mismatch_report(qt.scales.cpu().numpy(), ts, "W_dn^T scales"))
+    assert not msg, msg
+    ay = check_alpha(qy, host_amax(dy), "dY")
+    mi = sample_units(dy.shape[0], 62, 61)
+    ni = sample_units(Hd, 62, 62)
+    yr_enc = oracle.quantize_1d(host_f32(dy[torch.from_numpy(mi).to(DEV)]), alpha_in=ay)
+    check_rows(qy, mi, yr_enc, "dY")
+    bt = (tc[ni], None)
+    sc = np.array([[ts[oracle.sf_offset(int(n), j, D // 16, oracle.SF_TCGEN05)]
+                    for j in range(D // 16)] for n in ni], dtype=np.uint8)
+    yr, sr = oracle.gemm((yr_enc[0], yr_enc[1], ay, oracle.SF_ROWMAJOR),
+                         (bt[0], sc.reshape(-1), float(qd.alpha.cpu()[0]), oracle.SF_ROWMAJOR),
+                         len(mi), len(ni), D)
+    check_gemm(grid(dx, mi, ni), yr, sr, True, what="dX")

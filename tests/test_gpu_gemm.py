@@ -119,3 +119,24 @@ def test_ldo_larger_than_n():
     got = big.cpu().numpy()
     assert (np.abs(got[:, :144] - y) <= gemm_tolerance(y, s, False)).all()
     assert (got[:, 144:] == -7.0).all()  # untouched
+
+
+@pytest.mark.parametrize("T,Nout,Kin", [(200, 320, 256), (130, 3072, 400)])
+def test_dgrad_with_transposed_weight_codes(T, Nout, Kin):
+    """Data gradient dA = dO . W with W's 2D encoding transposed on the GPU
+    (no element re-quantized): the GEMM against the oracle's GEMM on the
+    oracle's transposed encoding, fp32 and bf16 outputs."""
+    do = synth.activation(13, 1, T, Nout)
+    w = synth.weight(13, 2, Nout, Kin)
+    qa = nv.quantize_1d(do.to(DEV))
+    qwt = nv.transpose_2d(nv.quantize_2d(w.to(DEV)))
+    aref = oracle.quantize_1d(to_oracle(do), sf_layout=oracle.SF_TCGEN05)
+    wref = oracle.quantize_2d(to_oracle(w), sf_layout=oracle.SF_TCGEN05)
+    tc, ts = oracle.transpose_2d(wref[0], wref[1], Nout, Kin, oracle.SF_TCGEN05, oracle.SF_TCGEN05)
+    assert_q_equal(qwt, (tc, ts, wref[2]), "W^T")
+    y, s = oracle_gemm_ref(aref, (tc, ts, wref[2]), T, Kin, Nout)
+    for dt in (torch.float32, torch.bfloat16):
+        got = nv.gemm(qa, qwt, out_dtype=dt).float().cpu().numpy().astype(np.float64)
+        tol = gemm_tolerance(y, s, dt == torch.bfloat16)
+        bad = np.argwhere(np.abs(got - y) > tol)
+        assert bad.size == 0, "%d outputs out of tolerance, first %s" % (len(bad), bad[0])

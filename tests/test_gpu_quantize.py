@@ -243,3 +243,20 @@ def test_window_gather_dequant(layout):
                 got = o.cpu().numpy().view(np.uint32)
                 want = d32[rows].view(np.uint32)
             assert np.array_equal(got, want), mismatch_report(got, want, "gather dequant")
+
+
+@pytest.mark.parametrize("rows,cols", [(144, 176), (160, 272), (64, 64)])
+@pytest.mark.parametrize("lin,lout", [(nv.NVFP4_SF_ROWMAJOR, nv.NVFP4_SF_ROWMAJOR),
+                                      (nv.NVFP4_SF_TCGEN05, nv.NVFP4_SF_TCGEN05),
+                                      (nv.NVFP4_SF_TCGEN05, nv.NVFP4_SF_ROWMAJOR)])
+def test_transpose_2d(rows, cols, lin, lout):
+    """The weight operand of the data-gradient GEMM: the transposed 2D
+    encoding, codes and scale bytes (padding included) bit for bit."""
+    w = synth.weight(12, 1, rows, cols)
+    q = nv.quantize_2d(w.to(DEV), sf_layout=lin)
+    t = nv.transpose_2d(q, sf_layout=lout)
+    ref = oracle.quantize_2d(to_oracle(w), sf_layout=lin)
+    assert_q_equal(q, ref, "W")
+    tc, ts = oracle.transpose_2d(ref[0], ref[1], rows, cols, lin, lout)
+    assert (t.rows, t.cols) == (cols, rows)
+    assert_q_equal(t, (tc, ts, ref[2]), "W^T")
