@@ -36,6 +36,24 @@ LAUNCHES_PER_STEP = 5
 CPU_MS, CPU_NS = 64, 128
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one QKV-shape
+# GEMM launch from an ncu capture (profiles/gemm_kernel_2sm_qkv_and_ffn.md),
+# valid only for the kernel source it was taken on.
+GEMM_TRAFFIC = {"source_sha256": None, "bytes_per_launch": None}
+
+
+def gemm_traffic():
+    import hashlib
+    src = os.path.join(ROOT, "nvfp4_block_scaled_20_b200", "csrc", "gemm.cu")
+    try:
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    if GEMM_TRAFFIC["source_sha256"] != digest:
+        return None
+    return GEMM_TRAFFIC["bytes_per_launch"]
+
+
 def peaks():
     """Roofline denominators from MEASURED_PEAKS.json (driver-written), else
     the pool's fallback measurement."""
@@ -409,7 +427,6 @@ def main():
     reps = max(20, min(args.steps, 200))
     part = {k: timed(graphs[k], reps)
             for k in ("amax_x", "pass2_x", "quant_x", "amax_w", "pass2_w", "quant_w", "gemm")}
-    clk = clocks.stop()
     assert nv.device_error(ws_g, stream) == 0
 
     step_ms_max = reduce_max(step_ms, world, dev)
@@ -444,6 +461,8 @@ def main():
         del graphs
         rows = measure_rows(nv, synth, torch, dev, stream, timed, pk, reps)
         graphs = None
+    # clocks sampled over every timed region (step, breakdown, rows)
+    clk = clocks.stop()
 
     e2e = None
     if not args.no_e2e:
@@ -466,7 +485,7 @@ def main():
                        "timing": "CUDA events around a CUDA-graph replay of the step, max over ranks"},
             "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1),
                          "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                         "frac": round(gemm_tflops / fp4_peak, 4), "traffic": None,
+                         "frac": round(gemm_tflops / fp4_peak, 4), "traffic": gemm_traffic(),
                          "kernel": "gemm_kernel<256> (tcgen05.mma kind::mxf4nvf4)",
                          "peak_source": "%s bf16 burst %.1f TFLOP/s x 4 (nominal dense FP4:BF16 "
                                         "ratio)" % (pk["source"], pk["bf16_tflops"])},

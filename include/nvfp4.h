@@ -203,7 +203,7 @@ NVFP4_API nvfp4_status nvfp4_quantize_1d_batched(const nvfp4_tensor_desc* descs,
  * framework's allocator that forbids side allocations, loops that must not
  * call cudaMalloc because it synchronizes the device, or C callers holding
  * only their tensors' raw pointers.  The per-tensor amax scratch is a fixed
- * array inside the library (about 80 KB on every GPU that loads it, kept
+ * array inside the library (about 115 KB on every GPU that loads it, kept
  * until the process exits); the call allocates and frees nothing.
  *   descs, n, dtype, qp: as nvfp4_quantize_1d_batched; block_axis must be 0
  *   and global_scale_in NULL.  n <= 64, else NVFP4_ERR_SHAPE.

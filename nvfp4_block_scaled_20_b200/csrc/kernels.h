@@ -10,7 +10,7 @@ namespace nvfp4 {
 constexpr int kMaxBatch = 64;  // tensors per batched launch (kernel parameter space)
 // Per-CTA partial maxima of the amax pass: at most this many CTAs per tensor,
 // one fp32 slot each in the workspace.
-constexpr int kMaxAmaxCtas = 320;
+constexpr int kMaxAmaxCtas = 448;
 
 struct QTensor {
   const void* x;

@@ -524,7 +524,7 @@ enum { kModeRows = 0, kModeCols = 1, kMode2D = 2 };
 // One CTA of the amax pass over tensor blockIdx.y: its partial maximum goes to
 // partials[t * kMaxAmaxCtas + blockIdx.x].
 template <typename T, int MODE, bool RHT>
-__global__ void __launch_bounds__(kThreads) amax_kernel(const __grid_constant__ QBatch p) {
+__global__ void __launch_bounds__(kThreads, 3) amax_kernel(const __grid_constant__ QBatch p) {
   const int t = blockIdx.y;
   // the row-axis mode reads its input as element pairs in both passes: its
   // rows need not satisfy the contiguous path's 32-byte alignment
@@ -660,35 +660,57 @@ __global__ void __launch_bounds__(kThreads) dequant_rows_kernel(const __grid_con
 
 // ------------------------------------------------------------------------
 // Transpose of a 2D (16x16-tile) encoding: the data-gradient GEMM's weight
-// operand.  A CTA moves 64 x 64 codes through shared memory (one byte per
-// code; rows padded to 68 bytes so the column reads hit 32 different banks)
-// and writes each output block's scale from its tile: output (c, b) takes
-// input (16 b, c / 16).  rows and cols are multiples of 16.
+// operand.  A CTA moves 64 rows x 256 codes through shared memory (one byte
+// per code; rows padded to 260 bytes): each thread loads 64 codes of one row
+// (four 8-byte loads in flight), then four threads write each output row's
+// 32 contiguous bytes;
+// each output block's scale comes from its tile: output (c, b) takes input
+// (16 b, c / 16).  rows and cols are multiples of 16.
+constexpr int kTrRows = 64, kTrCols = 256;
 __global__ void __launch_bounds__(kThreads)
     transpose_2d_kernel(const uint8_t* codes, const uint8_t* scales, int sf_in, int64_t rows,
                         int64_t cols, uint8_t* out_codes, uint8_t* out_scales, int sf_out) {
-  __shared__ uint8_t t[64][68];
-  const int64_t tiles_c = (cols + 63) / 64;
-  const int64_t ntiles = ((rows + 63) / 64) * tiles_c;
+  __shared__ __align__(16) uint8_t t[kTrRows][kTrCols + 4];
+  const int64_t tiles_c = (cols + kTrCols - 1) / kTrCols;
+  const int64_t ntiles = ((rows + kTrRows - 1) / kTrRows) * tiles_c;
   const int lr = threadIdx.x >> 2, part = threadIdx.x & 3;
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const int64_t r0 = (tile / tiles_c) * 64, c0 = (tile % tiles_c) * 64;
-    {  // thread: row r0 + lr, codes c0 + 16 part .. + 15
-      const int64_t r = r0 + lr, c = c0 + 16 * part;
-      uint2 w = make_uint2(0u, 0u);
-      if (r < rows && c < cols) w = __ldg(reinterpret_cast<const uint2*>(codes + r * (cols >> 1) + (c >> 1)));
+    const int64_t r0 = (tile / tiles_c) * kTrRows, c0 = (tile % tiles_c) * kTrCols;
+    {  // thread: row r0 + lr, codes c0 + 64 part .. + 63 (four 16-code chunks)
+      const int64_t r = r0 + lr;
+      uint2 w[4];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) t[lr][16 * part + i] = (uint8_t)(((i < 8 ? w.x : w.y) >> (4 * (i & 7))) & 0xFu);
+      for (int j = 0; j < 4; ++j) {
+        const int64_t c = c0 + 64 * part + 16 * j;
+        w[j] = (r < rows && c < cols)
+                   ? __ldg(reinterpret_cast<const uint2*>(codes + r * (cols >> 1) + (c >> 1)))
+                   : make_uint2(0u, 0u);
+      }
+      uint32_t* dst = reinterpret_cast<uint32_t*>(&t[lr][64 * part]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t v = h ? w[j].y : w[j].x;  // 8 codes, code i in bits 4i..4i+3
+          dst[4 * j + 2 * h] = (v & 0xFu) | ((v >> 4) & 0xFu) << 8 | ((v >> 8) & 0xFu) << 16 |
+                               ((v >> 12) & 0xFu) << 24;
+          dst[4 * j + 2 * h + 1] = ((v >> 16) & 0xFu) | ((v >> 20) & 0xFu) << 8 |
+                                   ((v >> 24) & 0xFu) << 16 | (v >> 28) << 24;
+        }
     }
     __syncthreads();
-    {  // thread: output row c0 + lr (input column), codes along rows r0 + 16 part .. + 15
-      const int64_t c = c0 + lr, r = r0 + 16 * part;
+    // output rows c0 .. c0 + 255 (input columns) in four passes of 64; the
+    // four threads of an output row write its 32 contiguous bytes
+#pragma unroll 1
+    for (int pass = 0; pass < kTrCols / 64; ++pass) {
+      const int lc = pass * 64 + lr, j = part;
+      const int64_t c = c0 + lc, r = r0 + 16 * j;
       if (c < cols && r < rows) {
         uint32_t lo = 0u, hi = 0u;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          lo |= (uint32_t)t[16 * part + i][lr] << (4 * i);
-          hi |= (uint32_t)t[16 * part + 8 + i][lr] << (4 * i);
+          lo |= (uint32_t)t[16 * j + i][lc] << (4 * i);
+          hi |= (uint32_t)t[16 * j + 8 + i][lc] << (4 * i);
         }
         *reinterpret_cast<uint2*>(out_codes + c * (rows >> 1) + (r >> 1)) = make_uint2(lo, hi);
         out_scales[sf_offset(c, r >> 4, rows >> 4, sf_out)] =
@@ -771,9 +793,9 @@ cudaError_t launch_mode(const QBatch& b, cudaStream_t s) {
   const uint64_t per_cta = (uint64_t)kThreads;
   int ga = 0;
   if (!b.gs_in) {
-    // amax pass: at most two CTAs per SM (up to four loads in flight per thread)
+    // amax pass: three CTAs per SM (eight 32-byte loads in flight per thread)
     uint64_t want = (units + 4 * per_cta - 1) / (4 * per_cta);
-    uint64_t cap = (uint64_t)num_sms() * 2;
+    uint64_t cap = (uint64_t)num_sms() * 3;
     if (cap > (uint64_t)kMaxAmaxCtas) cap = kMaxAmaxCtas;
     ga = (int)(want < 1 ? 1 : (want < cap ? want : cap));
     cudaError_t e = launch_ex(amax_kernel<T, MODE, RHT>, dim3(ga, b.n), s, false, b);
@@ -842,7 +864,8 @@ cudaError_t launch_dequantize_rows(const DQGather& g, cudaStream_t s) {
 cudaError_t launch_transpose_2d(const uint8_t* codes, const uint8_t* scales, int sf_in,
                                 int64_t rows, int64_t cols, uint8_t* out_codes,
                                 uint8_t* out_scales, int sf_out, cudaStream_t s) {
-  const uint64_t tiles = (uint64_t)((rows + 63) / 64) * (uint64_t)((cols + 63) / 64);
+  const uint64_t tiles = (uint64_t)((rows + kTrRows - 1) / kTrRows) *
+                         (uint64_t)((cols + kTrCols - 1) / kTrCols);
   const uint64_t cap = (uint64_t)num_sms() * 8;
   const int grid = (int)(tiles < cap ? (tiles < 1 ? 1 : tiles) : cap);
   transpose_2d_kernel<<<grid, kThreads, 0, s>>>(codes, scales, sf_in, rows, cols, out_codes,
