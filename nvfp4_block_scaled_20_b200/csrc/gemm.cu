@@ -59,7 +59,12 @@ constexpr int kBBytes = (BN / 2) * BK_BYTES;    // 16 KB: this CTA's half of B
 constexpr int kSfaBytes = 4 * 512;              // 4 atoms (128 rows x 16 blocks)
 constexpr int kSfbBytes = (BN / 128) * 4 * 512; // both 128-row bands of the tile
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 512 /*barriers*/;
+// epilogue staging: per epilogue warp two buffers of a 32-row x 16-column
+// output chunk (fp32 size), stored to global memory by TMA
+constexpr int kEpiChunkBytes = 32 * 16 * 4;
+constexpr int kEpiStageBytes = kEpiWarps * 2 * kEpiChunkBytes;
+constexpr int kSmemBytes =
+    kStages * kStageBytes + kEpiStageBytes + 1024 /*align*/ + 512 /*barriers*/;
 // tensor memory columns
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAcc1Col = 160;   // accumulator 0 at column 0, 1 at 160
@@ -154,6 +159,29 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(cluster_bar)
       : "memory");
+}
+// Tile store from this CTA's shared memory (dense box) to global memory;
+// rows and columns outside the tensor are clipped.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t c0,
+                                             int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          (uint64_t)map),
+      "r"(src), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// at most one committed store group still reading its shared memory
+__device__ __forceinline__ void bulk_wait_read_one() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
                                           uint32_t bar) {
@@ -274,8 +302,10 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mt
   nt = r / gm;
 }
 
-__device__ __forceinline__ void store16(const Params& p, int row, int col, const uint32_t r[16],
-                                        float scale) {
+// One lane's 16 accumulator columns -> x alpha_a*alpha_b, optional GELU ->
+// its row of the warp's staging chunk (32 rows x 16 columns, dense).
+__device__ __forceinline__ void stage16(const Params& p, uint8_t* chunk, int lane,
+                                        const uint32_t r[16], float scale) {
   float v[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
@@ -289,11 +319,11 @@ __device__ __forceinline__ void store16(const Params& p, int row, int col, const
       __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
       w[i] = *reinterpret_cast<uint32_t*>(&h);
     }
-    uint4* d4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + (int64_t)row * p.ldo + col);
+    uint4* d4 = reinterpret_cast<uint4*>(chunk + lane * 32);
     d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
     d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
   } else {
-    float4* d4 = reinterpret_cast<float4*>(static_cast<float*>(p.out) + (int64_t)row * p.ldo + col);
+    float4* d4 = reinterpret_cast<float4*>(chunk + lane * 64);
 #pragma unroll
     for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
   }
@@ -301,14 +331,15 @@ __device__ __forceinline__ void store16(const Params& p, int row, int col, const
 
 __global__ void __launch_bounds__(kNumThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ Params p) {
+                const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = smem;
   uint8_t* sB = sA + kStages * kABytes;
   uint8_t* sSFA = sB + kStages * kBBytes;
   uint8_t* sSFB = sSFA + kStages * kSfaBytes;
-  uint64_t* bars = (uint64_t*)(sSFB + kStages * kSfbBytes);
+  uint8_t* sEpi = sSFB + kStages * kSfbBytes;  // epilogue staging (1024-aligned)
+  uint64_t* bars = (uint64_t*)(sEpi + kEpiStageBytes);
   uint64_t* full = bars;                      // [kStages] codes of both CTAs landed (leader)
   uint64_t* sf_in = full + kStages;           // [kStages] this CTA's scale atoms landed
   uint64_t* empty = sf_in + kStages;          // [kStages] stage free: MMAs done + scales read
@@ -470,7 +501,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const int quad = warp & 3;     // TMEM lanes 32*quad .. 32*quad+31
     const int half = e >> 2;       // 0 / 1: first / second half of each column range
     const float scale = __fmul_rn(*p.a_alpha, *p.b_alpha);
-    uint32_t tile_i = 0;
+    uint8_t* my_stage = sEpi + e * 2 * kEpiChunkBytes;
+    uint32_t tile_i = 0, chunk_i = 0;
     for (int t = pair; t < num_tiles; t += num_pairs, ++tile_i) {
       const uint32_t b = tile_i & 1u, use = tile_i >> 1;
       int mt, nt;
@@ -483,7 +515,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       }
       tc_fence_after();
       const uint32_t t_acc = tmem + (b ? kAcc1Col : 0u) + ((uint32_t)(quad * 32) << 16);
-      const int row = m0 + quad * 32 + lane;
       const bool quad_live = m0 + quad * 32 < p.M;  // warp-uniform
       // The columns shared with the other accumulator (tile columns 160..255
       // of accumulator 0, 0..95 of accumulator 1) go first, split between
@@ -491,13 +522,25 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       const int ovl_c0 = b ? 0 : 256 - (int)kOvlCols;
       const int rest_c0 = b ? (int)kOvlCols : 0;
       constexpr int kOvlPer = (int)kOvlCols / 2, kRestPer = (256 - (int)kOvlCols) / 2;
+      // each 16-column chunk goes through one of the warp's two staging
+      // buffers and leaves as one TMA store (rows past M are clipped)
       auto drain = [&](int c0, int ncols) {
 #pragma unroll 1
         for (int c = c0; c < c0 + ncols; c += 16) {
           if (!quad_live || n0 + c >= p.N) continue;
+          uint8_t* chunk = my_stage + (chunk_i & 1u) * kEpiChunkBytes;
+          if (lane == 0) bulk_wait_read_one();  // this buffer's previous store has read it
+          __syncwarp();
           uint32_t r[16];
           tmem_ld16(t_acc + (uint32_t)c, r);
-          if (row < p.M) store16(p, row, n0 + c, r, scale);
+          stage16(p, chunk, lane, r, scale);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmOut, smem_u32(chunk), n0 + c, m0 + quad * 32);
+            bulk_commit();
+          }
+          ++chunk_i;
         }
       };
       drain(ovl_c0 + half * kOvlPer, kOvlPer);
@@ -509,6 +552,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_leader(smem_u32(&acc_empty[b]), leader);
     }
+    // every store has left shared memory and reached global memory
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ scale staging
     // Quadrant q's lanes get, per MMA k-block k of the stage: A columns
@@ -625,8 +671,27 @@ cudaLaunchConfig_t pair_config(dim3 grid, cudaStream_t s, cudaLaunchAttribute at
   return cfg;
 }
 
+// Output [M, N] (bf16 or fp32, row stride ldo elements), box = 16 columns x
+// 32 rows, dense in shared memory; stores clip at the tensor's edges.
+bool make_out_map(CUtensorMap* map, void* out, int64_t M, int64_t N, int64_t ldo, bool bf16) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t esz = bf16 ? 2 : 4;
+  cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+  cuuint64_t strides[1] = {(cuuint64_t)ldo * esz};
+  cuuint32_t box[2] = {16, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                  out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int launch_persistent(const GemmArgs& a, cudaStream_t s) {
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB, tmOut;
+  if (!make_out_map(&tmOut, a.out, a.M, a.N, a.ldo, a.out_bf16 != 0))
+    return (int)cudaErrorInvalidValue;
   if (!make_codes_map(&tmA, a.a_codes, a.M, a.K, BM)) return (int)cudaErrorInvalidValue;
   if (!make_codes_map(&tmB, a.b_codes, a.N, a.K, BN / 2)) return (int)cudaErrorInvalidValue;
   Params p;
@@ -659,7 +724,7 @@ int launch_persistent(const GemmArgs& a, cudaStream_t s) {
   const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
   cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = pair_config(dim3(2 * pairs), s, attr);
-  return (int)cudaLaunchKernelEx(&cfg, gemm_kernel, tmA, tmB, p);
+  return (int)cudaLaunchKernelEx(&cfg, gemm_kernel, tmA, tmB, tmOut, p);
 }
 
 }  // namespace
