@@ -11,14 +11,16 @@
 // memory and output rows [128 r, 128 r + 128) in tensor memory, so each SM
 // stores and serves only half of B -- the operand traffic through shared
 // memory per MMA is two thirds of a single-SM 128 x 256 tile's.
-//   warp 0       TMA producer (both CTAs): codes with the 2-SM form of
-//                cp.async.bulk.tensor (no multicast; completion counted on
-//                the leader CTA's barrier), scale atoms with cp.async.bulk
-//                into its own CTA, a 5-deep ring that runs ahead across tiles;
+//   warp 0       TMA producer (both CTAs): each CTA loads its own code tiles
+//                with the 2-SM form of cp.async.bulk.tensor (completion
+//                counted on the leader CTA's barrier) and its scale atoms
+//                with cp.async.bulk, a 5-deep ring that runs ahead across
+//                tiles;
 //   warp 1       allocates tensor memory (cta_group::2); in the leader CTA one
 //                thread issues the four MMAs (kind::mxf4nvf4, block16 scales,
-//                K = 64) of each stage; tcgen05.commit multicast to both CTAs
-//                releases ring stages and scale slots and signals accumulators;
+//                K = 64) of each stage; a tcgen05.commit that arrives in both
+//                CTAs releases ring stages and scale slots and signals the
+//                accumulators;
 //   warps 2..9   epilogue (both CTAs): tcgen05.ld of the CTA's 128 accumulator
 //                rows (two warps per 32-lane quadrant), x alpha_a*alpha_b,
 //                optional GELU(tanh), bf16 / fp32 stores;
@@ -150,8 +152,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
   }
 }
-// Tile load into this CTA's shared memory, completion counted on a barrier of
-// either CTA of the pair (2-SM form, no multicast).
+// Tile load into this CTA's own shared memory, completion counted on a
+// barrier of either CTA of the pair (2-SM form).
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int32_t c0,
                                                  int32_t c1, uint32_t cluster_bar) {
   asm volatile(
@@ -271,11 +273,13 @@ __device__ __forceinline__ float tanh_hw(float x) {
   asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
   return r;
 }
+// With fused multiply-adds: sqrt(2/pi) (y + 0.044715 y^3) = y (k0 + k0 k1 y^2)
+// and 0.5 y (1 + t) = 0.5 y t + 0.5 y (fp32 rounding, far inside the bound).
 __device__ __forceinline__ float gelu_tanh(float y) {
-  const float k0 = 0.7978845608028654f, k1 = 0.044715f;
-  const float y3 = __fmul_rn(__fmul_rn(y, y), y);
-  const float inner = __fmul_rn(k0, __fadd_rn(y, __fmul_rn(k1, y3)));
-  return __fmul_rn(__fmul_rn(0.5f, y), __fadd_rn(1.0f, tanh_hw(inner)));
+  const float k0 = 0.7978845608028654f, k01 = 0.7978845608028654f * 0.044715f;
+  const float inner = y * fmaf(k01, y * y, k0);
+  const float hy = 0.5f * y;
+  return fmaf(hy, tanh_hw(inner), hy);
 }
 
 struct Params {
