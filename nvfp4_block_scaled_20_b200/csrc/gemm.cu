@@ -230,6 +230,32 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t r[16]) {
       : "memory");
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// The load without its wait; the registers are valid only after tmem_wait16.
+__device__ __forceinline__ void tmem_ld16_async(uint32_t taddr, uint32_t r[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+// Waits for every tcgen05.ld of this thread (kWait) or only orders after an
+// earlier wait; either way r passes through the statement, so no use of it is
+// scheduled before the wait.
+#define NVFP4_TIE16(r)                                                                        \
+  "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),         \
+      "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), \
+      "+r"(r[14]), "+r"(r[15])
+template <bool kWait>
+__device__ __forceinline__ void tmem_wait16(uint32_t r[16]) {
+  if constexpr (kWait)
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : NVFP4_TIE16(r) : : "memory");
+  else
+    asm volatile("" : NVFP4_TIE16(r) : : "memory");
+}
+#undef NVFP4_TIE16
 // Tensor-memory stores of 16 consecutive 32-bit columns for the 32 lanes of
 // this warp's quadrant (taddr carries the quadrant's first lane).
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t r[16]) {
@@ -522,35 +548,55 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       const bool quad_live = m0 + quad * 32 < p.M;  // warp-uniform
       // The columns shared with the other accumulator (tile columns 160..255
       // of accumulator 0, 0..95 of accumulator 1) go first, split between
-      // the two warps of each quadrant; then the rest.
+      // the two warps of each quadrant: read into registers with one wait and
+      // released at once, since the next tile's MMAs wait for them; then
+      // staged and stored, then the rest.
       const int ovl_c0 = b ? 0 : 256 - (int)kOvlCols;
       const int rest_c0 = b ? (int)kOvlCols : 0;
       constexpr int kOvlPer = (int)kOvlCols / 2, kRestPer = (256 - (int)kOvlCols) / 2;
+      static_assert(kOvlPer == 48, "three 16-column chunks of shared columns per warp");
       // each 16-column chunk goes through one of the warp's two staging
       // buffers and leaves as one TMA store (rows past M are clipped)
+      auto store_chunk = [&](int c, const uint32_t r[16]) {
+        uint8_t* chunk = my_stage + (chunk_i & 1u) * kEpiChunkBytes;
+        if (lane == 0) bulk_wait_read_one();  // this buffer's previous store has read it
+        __syncwarp();
+        stage16(p, chunk, lane, r, scale);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmOut, smem_u32(chunk), n0 + c, m0 + quad * 32);
+          bulk_commit();
+        }
+        ++chunk_i;
+      };
       auto drain = [&](int c0, int ncols) {
 #pragma unroll 1
         for (int c = c0; c < c0 + ncols; c += 16) {
           if (!quad_live || n0 + c >= p.N) continue;
-          uint8_t* chunk = my_stage + (chunk_i & 1u) * kEpiChunkBytes;
-          if (lane == 0) bulk_wait_read_one();  // this buffer's previous store has read it
-          __syncwarp();
           uint32_t r[16];
           tmem_ld16(t_acc + (uint32_t)c, r);
-          stage16(p, chunk, lane, r, scale);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmOut, smem_u32(chunk), n0 + c, m0 + quad * 32);
-            bulk_commit();
-          }
-          ++chunk_i;
+          store_chunk(c, r);
         }
       };
-      drain(ovl_c0 + half * kOvlPer, kOvlPer);
+      const int oc = ovl_c0 + half * kOvlPer;
+      uint32_t o0[16], o1[16], o2[16];
+      if (quad_live) {
+        tmem_ld16_async(t_acc + (uint32_t)oc, o0);
+        tmem_ld16_async(t_acc + (uint32_t)(oc + 16), o1);
+        tmem_ld16_async(t_acc + (uint32_t)(oc + 32), o2);
+        tmem_wait16<true>(o0);
+        tmem_wait16<false>(o1);
+        tmem_wait16<false>(o2);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_leader(smem_u32(ovl_free), leader);
+      if (quad_live) {
+        if (n0 + oc < p.N) store_chunk(oc, o0);
+        if (n0 + oc + 16 < p.N) store_chunk(oc + 16, o1);
+        if (n0 + oc + 32 < p.N) store_chunk(oc + 32, o2);
+      }
       drain(rest_c0 + half * kRestPer, kRestPer);
       tc_fence_before();
       __syncwarp();
