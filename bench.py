@@ -677,39 +677,69 @@ def measure_rows(nv, synth, torch, dev, stream, timed, pk, reps):
 
 def measure_e2e(nv, torch, dev, stream, x, w, qa, qb, ws_a, ws_b, ws_g, args, world):
     """Same step through the public API with the inputs copied from pinned host
-    memory and the bf16 result copied back, every step."""
+    memory and the bf16 result copied back, every step.  Steps are pipelined
+    over three streams (inputs in, compute, result out; device buffers double
+    buffered), so step i's host-to-device copies overlap step i-1's compute
+    and step i-2's device-to-host copy; every step still moves all its bytes
+    inside the timed region."""
     hx = x.cpu().pin_memory()
     hw = w.cpu().pin_memory()
-    hy = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-    dx = torch.empty_like(x)
-    dw = torch.empty_like(w)
-    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    hy = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    dx = [torch.empty_like(x) for _ in range(2)]
+    dw = [torch.empty_like(w) for _ in range(2)]
+    y = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev = lambda: [torch.cuda.Event() for _ in range(2)]  # noqa: E731
+    ev_in, ev_used, ev_done, ev_out = ev(), ev(), ev(), ev()
     steps = max(3, min(args.steps, 50))
 
-    def one():
-        dx.copy_(hx, non_blocking=True)
-        dw.copy_(hw, non_blocking=True)
-        nv.quantize_1d(dx, out=qa, ws=ws_a, stream=stream)
-        nv.quantize_2d(dw, out=qb, ws=ws_b, stream=stream)
-        nv.gemm(qa, qb, out=y, ws=ws_g, stream=stream)
-        hy.copy_(y, non_blocking=True)
+    def one(i):
+        b = i % 2
+        # inputs: wait until step i-2's compute has read buffer b
+        if i >= 2:
+            s_in.wait_event(ev_used[b])
+        with torch.cuda.stream(s_in):
+            dx[b].copy_(hx, non_blocking=True)
+            dw[b].copy_(hw, non_blocking=True)
+        ev_in[b].record(s_in)
+        # compute: inputs landed, and step i-2's result has left y[b]
+        stream.wait_event(ev_in[b])
+        if i >= 2:
+            stream.wait_event(ev_out[b])
+        nv.quantize_1d(dx[b], out=qa, ws=ws_a, stream=stream)
+        nv.quantize_2d(dw[b], out=qb, ws=ws_b, stream=stream)
+        ev_used[b].record(stream)
+        nv.gemm(qa, qb, out=y[b], ws=ws_g, stream=stream)
+        ev_done[b].record(stream)
+        # result out
+        s_out.wait_event(ev_done[b])
+        with torch.cuda.stream(s_out):
+            hy[b].copy_(y[b], non_blocking=True)
+        ev_out[b].record(s_out)
 
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            one()
-    stream.synchronize()
+    def run(n):
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        s_in.wait_event(start)
+        s_out.wait_event(start)
+        for i in range(n):
+            one(i)
+        stream.wait_event(ev_out[(n - 1) % 2])
+        stream.wait_event(ev_out[n % 2])
+        end.record(stream)
+        return start, end
+
+    run(3)
+    torch.cuda.synchronize(dev)
     barrier(world)
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        s.record(stream)
-        for _ in range(steps):
-            one()
-        e.record(stream)
-    stream.synchronize()
+    s, e = run(steps)
+    torch.cuda.synchronize(dev)
     ms = reduce_max(s.elapsed_time(e) / steps, world, dev)
     return {"value": world * 2.0 * M * N * K / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "ms_per_step": ms, "h2d_bytes_per_step": x.numel() * 2 + w.numel() * 2,
-            "d2h_bytes_per_step": M * N * 2}
+            "d2h_bytes_per_step": M * N * 2,
+            "pipelined": "h2d / compute / d2h on three streams, device buffers double buffered"}
 
 
 if __name__ == "__main__":

@@ -448,15 +448,36 @@ __device__ void encode_2d(const QTensor& q, float alpha, const QBatch& p, uint2*
     load16(x + (int64_t)r * q.ld + (int64_t)kb * 16, v);
     redo_block(v, it.y, ctx, fos, q.codes + (int64_t)r * (q.cols >> 1) + (int64_t)kb * 8, nullptr);
   };
-  WarpQueue wq{qbuf, 0u};
-  for (uint32_t u = blockIdx.x * warps + (threadIdx.x >> 5); u < nunits; u += gridDim.x * warps) {
+  // this lane's block of unit u: row r, block column kb (false past the last column)
+  auto block_of = [&](uint32_t u, int64_t& r, uint32_t& kb) {
     const uint32_t tr = fastdiv(u, div), tp = u - tr * npair;
-    const int64_t r = (int64_t)tr * 16 + (lane & 15);
-    const uint32_t kb = tp * 2 + (lane >> 4);
-    const bool valid = kb < kbpr;
+    r = (int64_t)tr * 16 + (lane & 15);
+    kb = tp * 2 + (lane >> 4);
+    return kb < kbpr;
+  };
+  WarpQueue wq{qbuf, 0u};
+  const uint32_t ustride = gridDim.x * warps;
+  uint32_t u = blockIdx.x * warps + (threadIdx.x >> 5);
+  // the next unit's block is loaded before the current one is encoded
+  RawBlock<T> next;
+  if (u < nunits) {
+    int64_t r;
+    uint32_t kb;
+    if (block_of(u, r, kb)) next.load(x + r * q.ld + (int64_t)kb * 16);
+  }
+  for (; u < nunits; u += ustride) {
+    int64_t r;
+    uint32_t kb;
+    const bool valid = block_of(u, r, kb);
+    const RawBlock<T> cur = next;
+    if (u + ustride < nunits) {
+      int64_t rn;
+      uint32_t kbn;
+      if (block_of(u + ustride, rn, kbn)) next.load(x + rn * q.ld + (int64_t)kbn * 16);
+    }
     float v[16];
     if (valid) {
-      load16(x + r * q.ld + (int64_t)kb * 16, v);
+      cur.widen(v);
     } else {
 #pragma unroll
       for (int i = 0; i < 16; ++i) v[i] = 0.0f;
