@@ -39,7 +39,8 @@ CPU_MS, CPU_NS = 64, 128
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one QKV-shape
 # GEMM launch from an ncu capture (profiles/gemm_kernel_2sm_qkv_and_ffn.md),
 # valid only for the kernel source it was taken on.
-GEMM_TRAFFIC = {"source_sha256": None, "bytes_per_launch": None}
+GEMM_TRAFFIC = {"source_sha256": "168fb4235c29b87813e02abca004d94d89bdaa83efa2e3d15356fca6914bc170",
+                "bytes_per_launch": 20541440 + 4496896}
 
 
 def gemm_traffic():
@@ -486,7 +487,7 @@ def main():
             "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1),
                          "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                          "frac": round(gemm_tflops / fp4_peak, 4), "traffic": gemm_traffic(),
-                         "kernel": "gemm_kernel<256> (tcgen05.mma kind::mxf4nvf4)",
+                         "kernel": "gemm_kernel (CTA-pair tcgen05.mma kind::mxf4nvf4)",
                          "peak_source": "%s bf16 burst %.1f TFLOP/s x 4 (nominal dense FP4:BF16 "
                                         "ratio)" % (pk["source"], pk["bf16_tflops"])},
             "breakdown": breakdown,
