@@ -30,8 +30,9 @@ M, N, K = 2640, 9216, 3072
 WORKLOAD = "DiT QKV projection W4A4: X bf16 [2640x3072] (1% Student-t(3)x8 channels), " \
            "W bf16 [9216x3072] N(0,0.02); 1D act + 2D weight NVFP4, 4-vs-6 on; Y bf16 [2640x9216]"
 FLUSH_BYTES = 256 << 20
-# our kernels per step: amax + encode for X, amax + encode for W, the GEMM
-LAUNCHES_PER_STEP = 5
+# our kernels per step: one amax and one encode launch for X and W together
+# (nvfp4_quantize_mixed), the GEMM
+LAUNCHES_PER_STEP = 3
 # CPU-oracle sample: the first rows of the same workload
 CPU_MS, CPU_NS = 64, 128
 
@@ -227,7 +228,7 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------ ncu cases
 PROFILE_CASES = {
-    "qkv_step": "DiT QKV step: quantize X [2640, 3072], quantize W [9216, 3072], GEMM",
+    "qkv_step": "DiT QKV step: quantize X [2640, 3072] (1D) and W [9216, 3072] (2D) in one mixed call, GEMM",
     "h_quantize": "1D quantize of an FFN-hidden-sized bf16 [8192, 14336]: amax + encode, "
                   "then encode alone (global scale given)",
     "w_quantize_2d": "2D quantize of W_up [14336, 3072]",
@@ -253,7 +254,8 @@ def run_profile_case(name, reps=3):
         x, w = synth.qkv_linear(dev)
 
         def run():
-            nv.gemm(nv.quantize_1d(x, ws=ws), nv.quantize_2d(w, ws=ws), ws=ws)
+            qx, qw = nv.quantize_mixed([x, w], [False, True], ws=ws)
+            nv.gemm(qx, qw, ws=ws)
     elif name == "h_quantize":
         h = synth.activation(2, 9, 8192, 14336, device=dev)
         qh = nv.quantize_1d(h, ws=ws)
@@ -344,6 +346,7 @@ def main():
     qb = nv.QTensor(*nv._alloc_q(N, K, nv.NVFP4_SF_TCGEN05, dev), N, K, nv.NVFP4_SF_TCGEN05)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     ws_a, ws_b, ws_g = nv.workspace(1, dev), nv.workspace(1, dev), nv.workspace(0, dev)
+    ws_xw = nv.workspace(2, dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_sink = torch.empty((), dtype=torch.float32, device=dev)
@@ -353,6 +356,9 @@ def main():
         # one so the next kernel does not pay for writing back dirty lines
         flush.zero_()
         torch.sum(flush_rd, dim=0, out=flush_sink)
+
+    def quant_xw():
+        nv.quantize_mixed([x, w], [False, True], outs=[qa, qb], ws=ws_xw, stream=stream)
 
     def quant_x():
         nv.quantize_1d(x, out=qa, ws=ws_a, stream=stream)
@@ -376,8 +382,7 @@ def main():
         nv.gemm(qa, qb, out=y, ws=ws_g, stream=stream)
 
     def step():
-        quant_x()
-        quant_w()
+        quant_xw()
         gemm()
 
     # warm-up (also sets kernel attributes before graph capture)
@@ -395,7 +400,8 @@ def main():
 
     graphs = {"step": capture(step), "amax_x": capture(amax_x), "pass2_x": capture(pass2_x),
               "amax_w": capture(amax_w), "pass2_w": capture(pass2_w), "gemm": capture(gemm),
-              "quant_x": capture(quant_x), "quant_w": capture(quant_w)}
+              "quant_x": capture(quant_x), "quant_w": capture(quant_w),
+              "quant_xw": capture(quant_xw)}
 
     def timed(g, reps):
         """Mean device time (ms) of one graph replay, L2 flushed before each."""
@@ -427,7 +433,8 @@ def main():
     # per-kernel breakdown (same protocol)
     reps = max(20, min(args.steps, 200))
     part = {k: timed(graphs[k], reps)
-            for k in ("amax_x", "pass2_x", "quant_x", "amax_w", "pass2_w", "quant_w", "gemm")}
+            for k in ("amax_x", "pass2_x", "quant_x", "amax_w", "pass2_w", "quant_w", "quant_xw",
+                      "gemm")}
     assert nv.device_error(ws_g, stream) == 0
 
     step_ms_max = reduce_max(step_ms, world, dev)
@@ -446,15 +453,18 @@ def main():
     breakdown = {
         "gemm": {"ms": round(part["gemm"], 5), "TFLOP/s": round(gemm_tflops, 1),
                  "frac_fp4_peak": round(gemm_tflops / fp4_peak, 3)},
+        "quantize_xw_mixed": gbs((4 + q_out) * (M + N) * K, part["quant_xw"]),
         "quantize_x": gbs((4 + q_out) * M * K, part["quant_x"]),
         "quantize_w": gbs((4 + q_out) * N * K, part["quant_w"]),
         "amax_only_x": gbs(2 * M * K, part["amax_x"]),
         "encode_only_x": gbs((2 + q_out) * M * K, part["pass2_x"]),
         "amax_only_w": gbs(2 * N * K, part["amax_w"]),
         "encode_only_w": gbs((2 + q_out) * N * K, part["pass2_w"]),
-        "note": "quantize_* is the fused amax + encode launch of the step, counted at the "
-                "algorithmic two-read bytes (4 + 0.5625 B/element); X (16 MB) and W (57 MB) fit in "
-                "L2, so its second read is served from L2.  Each line is timed after an L2 flush.",
+        "note": "quantize_xw_mixed is the step's quantization: one amax and one encode launch "
+                "for X (1D) and W (2D); quantize_x / quantize_w are the single-tensor calls "
+                "(amax + encode each).  All counted at the algorithmic two-read bytes "
+                "(4 + 0.5625 B/element); X (16 MB) and W (57 MB) fit in L2, so the second read is "
+                "served from L2.  Each line is timed after an L2 flush.",
     }
 
     rows = None
@@ -467,7 +477,7 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(nv, torch, dev, stream, x, w, qa, qb, ws_a, ws_b, ws_g, args, world)
+        e2e = measure_e2e(nv, torch, dev, stream, x, w, qa, qb, ws_xw, ws_g, args, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -676,7 +686,7 @@ def measure_rows(nv, synth, torch, dev, stream, timed, pk, reps):
     return out
 
 
-def measure_e2e(nv, torch, dev, stream, x, w, qa, qb, ws_a, ws_b, ws_g, args, world):
+def measure_e2e(nv, torch, dev, stream, x, w, qa, qb, ws_xw, ws_g, args, world):
     """Same step through the public API with the inputs copied from pinned host
     memory and the bf16 result copied back, every step.  Steps are pipelined
     over three streams (inputs in, compute, result out; device buffers double
@@ -707,8 +717,7 @@ def measure_e2e(nv, torch, dev, stream, x, w, qa, qb, ws_a, ws_b, ws_g, args, wo
         stream.wait_event(ev_in[b])
         if i >= 2:
             stream.wait_event(ev_out[b])
-        nv.quantize_1d(dx[b], out=qa, ws=ws_a, stream=stream)
-        nv.quantize_2d(dw[b], out=qb, ws=ws_b, stream=stream)
+        nv.quantize_mixed([dx[b], dw[b]], [False, True], outs=[qa, qb], ws=ws_xw, stream=stream)
         ev_used[b].record(stream)
         nv.gemm(qa, qb, out=y[b], ws=ws_g, stream=stream)
         ev_done[b].record(stream)

@@ -197,6 +197,30 @@ NVFP4_API nvfp4_status nvfp4_quantize_1d_batched(const nvfp4_tensor_desc* descs,
                                        void* workspace,
                                        size_t workspace_bytes, void* stream);
 
+/* Mixed quantization: the operands of W4A4 linear layers -- 1D activations
+ * and 2D weights (explainer, "NVFP4 training recipe for AR training": 1D
+ * blocks for activations and gradients, 16x16 blocks for weights) -- in one
+ * amax launch and one encode launch for all tensors, the GPU's CTAs split
+ * between them in proportion to their work.  Codes, scales and global
+ * scales are identical to nvfp4_quantize_1d / nvfp4_quantize_2d on each
+ * tensor (the split changes only which CTA does what).
+ *   descs[i]   x, codes, scales, global_scale, rows, cols, ld as in the
+ *              single-tensor calls (HOST array of n).
+ *   two_d[i]   HOST array of n: 0 = 1D blocks along cols, 1 = 16x16 tiles.
+ *   dtype      one input dtype for all tensors.
+ *   qp         four_over_six and sf_layout apply to all; rht_enable and
+ *              block_axis must be 0 and global_scale_in NULL (each tensor
+ *              gets the global scale of its own amax).
+ * n <= 64 (else NVFP4_ERR_SHAPE); shape and alignment rules per tensor as
+ * in the single-tensor calls; an empty tensor (rows or cols 0) only gets
+ * its global scale, 1.0 (its codes and scales may be NULL).
+ * Workspace: nvfp4_workspace_bytes(n). */
+NVFP4_API nvfp4_status nvfp4_quantize_mixed(const nvfp4_tensor_desc* descs,
+                                  const int32_t* two_d, int32_t n,
+                                  int32_t dtype, const nvfp4_qparams* qp,
+                                  void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
 /* Batched 1D quantization that takes no workspace (the paper has no
  * counterpart; this is a library convenience).  For callers that cannot
  * allocate device memory or pass a workspace: code running inside another

@@ -15,6 +15,7 @@ from .capi import (NVFP4_BF16, NVFP4_EPI_GELU_TANH, NVFP4_EPI_NONE, NVFP4_F32,  
                    NVFP4_SF_ROWMAJOR, NVFP4_SF_TCGEN05, NVFP4Error)
 
 __all__ = ["QTensor", "quantize_1d", "quantize_2d", "global_scale", "quantize_1d_batched",
+           "quantize_mixed",
            "dequantize", "dequantize_rows", "window_row_ranges", "transpose_2d", "gemm", "rht16", "workspace",
            "device_error", "capi"]
 
@@ -135,6 +136,30 @@ def quantize_1d_batched(xs, four_over_six=True, sf_layout=NVFP4_SF_ROWMAJOR, ws=
     st = capi.nvfp4_quantize_1d_batched(descs, n, _dtype_code(xs[0]), qp, ws.data_ptr(),
                                         ws.numel(), _stream(stream))
     capi.check("nvfp4_quantize_1d_batched", st)
+    return outs
+
+
+def quantize_mixed(xs, two_d, four_over_six=True, sf_layout=NVFP4_SF_TCGEN05, ws=None,
+                   outs=None, stream=None):
+    """One nvfp4_quantize_mixed call: xs[i] quantized 1D (two_d[i] false) or
+    in 16x16 tiles (true), each with the global scale of its own amax."""
+    import ctypes
+    n = len(xs)
+    if outs is None:
+        outs = [QTensor(*_alloc_q(x.shape[0], x.shape[1], sf_layout, x.device), x.shape[0],
+                        x.shape[1], sf_layout) for x in xs]
+    ws = workspace(n, xs[0].device) if ws is None else ws
+    descs = (capi.nvfp4_tensor_desc * n)()
+    flags = (ctypes.c_int32 * n)()
+    for i, (x, q) in enumerate(zip(xs, outs)):
+        descs[i] = capi.nvfp4_tensor_desc(x.data_ptr(), None, q.codes.data_ptr(),
+                                          q.scales.data_ptr(), q.alpha.data_ptr(), x.shape[0],
+                                          x.shape[1], x.stride(0))
+        flags[i] = 1 if two_d[i] else 0
+    qp = _qparams(four_over_six, 0, 0, 0, sf_layout, None)
+    st = capi.nvfp4_quantize_mixed(descs, flags, n, _dtype_code(xs[0]), qp, ws.data_ptr(),
+                                   ws.numel(), _stream(stream))
+    capi.check("nvfp4_quantize_mixed", st)
     return outs
 
 

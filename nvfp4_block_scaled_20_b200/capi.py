@@ -21,7 +21,7 @@ NVFP4_EPI_NONE, NVFP4_EPI_GELU_TANH = 0, 1
 
 EXPORTED = [
     "nvfp4_workspace_bytes", "nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_global_scale",
-    "nvfp4_quantize_1d", "nvfp4_quantize_2d", "nvfp4_quantize_1d_batched",
+    "nvfp4_quantize_1d", "nvfp4_quantize_2d", "nvfp4_quantize_1d_batched", "nvfp4_quantize_mixed",
     "nvfp4_quantize_1d_batched_noalloc", "nvfp4_dequantize", "nvfp4_dequantize_rows",
     "nvfp4_transpose_2d",
     "nvfp4_gemm", "nvfp4_rht16", "nvfp4_get_device_error", "nvfp4_status_string",
@@ -61,6 +61,8 @@ _SIGS = {
     "nvfp4_quantize_1d": (_I32, [_V, _I32, _I64, _I64, _I64, _QP, _V, _V, _V, _V, _SZ, _V]),
     "nvfp4_quantize_2d": (_I32, [_V, _I32, _I64, _I64, _I64, _QP, _V, _V, _V, _V, _SZ, _V]),
     "nvfp4_quantize_1d_batched": (_I32, [_TD, _I32, _I32, _QP, _V, _SZ, _V]),
+    "nvfp4_quantize_mixed": (_I32, [_TD, ctypes.POINTER(ctypes.c_int32), _I32, _I32, _QP, _V, _SZ,
+                                    _V]),
     "nvfp4_quantize_1d_batched_noalloc": (_I32, [_TD, _I32, _I32, _QP, _V]),
     "nvfp4_dequantize": (_I32, [_TD, _I32, _I32, _I32, _V]),
     "nvfp4_transpose_2d": (_I32, [_V, _V, _I32, _I64, _I64, _V, _V, _I32, _V]),
@@ -128,6 +130,11 @@ def nvfp4_quantize_2d(x, dtype, rows, cols, ld, qp, codes, scales, gs_out, ws, w
 
 def nvfp4_quantize_1d_batched(descs, n, dtype, qp, ws, ws_bytes, stream):
     return _call("nvfp4_quantize_1d_batched", descs, n, dtype, ctypes.byref(qp), ws, ws_bytes,
+                 stream)
+
+
+def nvfp4_quantize_mixed(descs, two_d, n, dtype, qp, ws, ws_bytes, stream):
+    return _call("nvfp4_quantize_mixed", descs, two_d, n, dtype, ctypes.byref(qp), ws, ws_bytes,
                  stream)
 
 

@@ -174,6 +174,39 @@ nvfp4_status nvfp4_quantize_1d_batched(const nvfp4_tensor_desc* descs, int32_t n
   return NVFP4_OK;
 }
 
+nvfp4_status nvfp4_quantize_mixed(const nvfp4_tensor_desc* descs, const int32_t* two_d,
+                                  int32_t n, int32_t dtype, const nvfp4_qparams* qp, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  if (!descs || !two_d || n < 0) return NVFP4_ERR_INVALID_ARG;
+  if (n > kMaxBatch) return NVFP4_ERR_SHAPE;
+  nvfp4_status st = check_qparams(qp, true);  // block_axis 0, no RHT
+  if (st != NVFP4_OK) return st;
+  if (qp->global_scale_in) return NVFP4_ERR_INVALID_ARG;
+  if (!dtype_ok(dtype)) return NVFP4_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < n; ++i) {
+    const nvfp4_tensor_desc& d = descs[i];
+    if (two_d[i] != 0 && two_d[i] != 1) return NVFP4_ERR_INVALID_ARG;
+    st = check_input(d.x, dtype, d.rows, d.cols, d.ld, 0, two_d[i] != 0);
+    if (st != NVFP4_OK) return st;
+    // an empty tensor only receives its global scale (1.0)
+    const bool empty = d.rows == 0 || d.cols == 0;
+    if ((!empty && (!d.codes || !d.scales)) || !d.global_scale) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(d.codes, 16) || !aligned(d.scales, 4) || !aligned(d.global_scale, 4))
+      return NVFP4_ERR_ALIGN;
+  }
+  if (!ws || ws_bytes < nvfp4_workspace_bytes(n)) return NVFP4_ERR_WORKSPACE;
+  if (n == 0) return NVFP4_OK;
+  QBatch b;
+  fill_batch_common(b, dtype, qp, ws);
+  b.n = n;
+  for (int32_t i = 0; i < n; ++i) {
+    const nvfp4_tensor_desc& d = descs[i];
+    b.t[i] = QTensor{d.x, d.codes, d.scales, d.global_scale, d.rows, d.cols, d.ld};
+    b.two_d_of[i] = (int8_t)two_d[i];
+  }
+  return cuda_status(launch_quantize_mixed(b, S(stream)));
+}
+
 nvfp4_status nvfp4_dequantize(const nvfp4_tensor_desc* descs, int32_t n, int32_t out_dtype,
                               int32_t sf_layout, void* stream) {
   if (!descs || n < 0 || !dtype_ok(out_dtype)) return NVFP4_ERR_INVALID_ARG;

@@ -36,6 +36,11 @@ struct QBatch {
   const float* gs_in;   // device; nullptr => from the amax pass
   float* partials;      // device, kMaxAmaxCtas slots per tensor (amax pass output)
   uint32_t* err;        // device error word
+  // Mixed launch (launch_quantize_mixed): 1D row-block and 2D tensors in one
+  // 1D grid per pass; tensor i owns blockIdx.x in [end[i-1], end[i]).
+  int32_t amax_end[kMaxBatch];
+  int32_t enc_end[kMaxBatch];
+  int8_t two_d_of[kMaxBatch];  // 1: tensor i is quantized in 16x16 tiles
 };
 
 struct DQTensor {
@@ -87,6 +92,11 @@ int num_sms();
 // global scale; only the encode kernel when gs_in is given, only the amax
 // kernel and a finalize kernel when amax_only is set.
 cudaError_t launch_quantize(const QBatch& b, cudaStream_t s);
+// 1D (block_axis 0, no RHT) and 2D tensors of one dtype, each with its own
+// global scale from its amax: one amax launch and one encode launch for all,
+// CTAs split between the tensors in proportion to their work.  Results equal
+// the per-tensor launches'.  Fills the CTA ranges of b.
+cudaError_t launch_quantize_mixed(QBatch& b, cudaStream_t s);
 cudaError_t launch_dequantize(const DQBatch& b, cudaStream_t s);
 cudaError_t launch_dequantize_rows(const DQGather& g, cudaStream_t s);
 cudaError_t launch_transpose_2d(const uint8_t* codes, const uint8_t* scales, int sf_in,

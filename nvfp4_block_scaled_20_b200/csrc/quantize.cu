@@ -73,6 +73,13 @@ __device__ float reduce_partials(const float* part, int ga) {
   return s_m;
 }
 
+// The CTAs of a launch that work on one tensor: cta-th of ncta.  A launch
+// over one tensor (or one tensor per blockIdx.y) uses (blockIdx.x,
+// gridDim.x); a mixed launch gives each tensor a range of blockIdx.x.
+struct Slice {
+  uint32_t cta, ncta;
+};
+
 // ------------------------------------------------------------------------
 // Amax pass.
 
@@ -80,13 +87,13 @@ __device__ float reduce_partials(const float* part, int ga) {
 // 32-byte loads in flight per thread (enough bytes in flight per SM to cover
 // the HBM latency at two CTAs per SM).
 constexpr int kAmaxDepth = 8;
-__device__ float amax_rows_bf16_raw(const QTensor& q) {
+__device__ float amax_rows_bf16_raw(const QTensor& q, const Slice sl) {
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(q.x);
   const uint32_t kbpr = (uint32_t)(q.cols >> 4);
   const uint64_t nblk = (uint64_t)q.rows * kbpr;
-  const uint64_t stride = (uint64_t)gridDim.x * kThreads;
+  const uint64_t stride = (uint64_t)sl.ncta * kThreads;
   uint32_t m2 = 0u;
-  for (uint64_t u = (uint64_t)blockIdx.x * kThreads + threadIdx.x; u < nblk; u += kAmaxDepth * stride) {
+  for (uint64_t u = (uint64_t)sl.cta * kThreads + threadIdx.x; u < nblk; u += kAmaxDepth * stride) {
     uint32_t w[kAmaxDepth][8];
 #pragma unroll
     for (int j = 0; j < kAmaxDepth; ++j) {
@@ -108,15 +115,15 @@ __device__ float amax_rows_bf16_raw(const QTensor& q) {
 }
 
 template <typename T, bool RHT>
-__device__ float amax_rows(const QTensor& q, uint32_t mask) {
-  if constexpr (std::is_same<T, __nv_bfloat16>::value && !RHT) return amax_rows_bf16_raw(q);
+__device__ float amax_rows(const QTensor& q, uint32_t mask, const Slice sl) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value && !RHT) return amax_rows_bf16_raw(q, sl);
   const T* x = static_cast<const T*>(q.x);
   const uint32_t kbpr = (uint32_t)(q.cols >> 4);
   const uint64_t nblk = (uint64_t)q.rows * kbpr;
-  const uint64_t stride = (uint64_t)gridDim.x * kThreads;
+  const uint64_t stride = (uint64_t)sl.ncta * kThreads;
   float m = 0.0f;
   // two blocks per thread per trip, both loads issued before any use
-  for (uint64_t u = (uint64_t)blockIdx.x * kThreads + threadIdx.x; u < nblk; u += 2 * stride) {
+  for (uint64_t u = (uint64_t)sl.cta * kThreads + threadIdx.x; u < nblk; u += 2 * stride) {
     float v[2][16];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -183,14 +190,14 @@ template <> struct RawPair<float> {
 // == 0 and cols even for this mode), with the RHT applied along rows when
 // enabled; two units' loads in flight per thread.
 template <typename T, bool RHT>
-__device__ float amax_cols(const QTensor& q, uint32_t mask) {
+__device__ float amax_cols(const QTensor& q, uint32_t mask, const Slice sl) {
   const T* x = static_cast<const T*>(q.x);
   const uint32_t ncp = (uint32_t)(q.cols >> 1);
   const uint32_t nunits = ncp * (uint32_t)(q.rows >> 4);
   const FastDiv div = make_fastdiv(ncp);
-  const uint32_t stride = gridDim.x * kThreads;
+  const uint32_t stride = sl.ncta * kThreads;
   float m = 0.0f;
-  for (uint32_t u = blockIdx.x * kThreads + threadIdx.x; u < nunits; u += 2 * stride) {
+  for (uint32_t u = sl.cta * kThreads + threadIdx.x; u < nunits; u += 2 * stride) {
     RawPair<T> raw[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -217,11 +224,11 @@ __device__ float amax_cols(const QTensor& q, uint32_t mask) {
 }
 
 // Zero the padding entries of a tcgen05-layout scale buffer.
-__device__ void zero_sf_padding(uint8_t* sf, int64_t rows, int64_t kbpr) {
+__device__ void zero_sf_padding(uint8_t* sf, int64_t rows, int64_t kbpr, const Slice sl) {
   const int64_t rows_pad = (rows + 127) & ~int64_t(127);
   const int64_t kb_pad = (kbpr + 3) & ~int64_t(3);
-  const int64_t tid = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  const int64_t step = (int64_t)gridDim.x * kThreads;
+  const int64_t tid = (int64_t)sl.cta * kThreads + threadIdx.x;
+  const int64_t step = (int64_t)sl.ncta * kThreads;
   const int64_t n1 = (rows_pad - rows) * kb_pad;  // whole padding rows
   for (int64_t i = tid; i < n1; i += step) {
     const int64_t r = rows + i / kb_pad, kb = i % kb_pad;
@@ -307,14 +314,15 @@ __device__ __forceinline__ void redo_block(const float v[16], uint32_t code, con
 // over blocks, the next block's load issued before the current one is
 // encoded.
 template <typename T, bool RHT>
-__device__ void encode_rows(const QTensor& q, float alpha, const QBatch& p, uint2* qbuf) {
+__device__ void encode_rows(const QTensor& q, float alpha, const QBatch& p, uint2* qbuf,
+                            const Slice sl) {
   const T* x = static_cast<const T*>(q.x);
   const uint32_t kbpr = (uint32_t)(q.cols >> 4);
   const uint32_t nblk = (uint32_t)q.rows * kbpr;  // < 2^32, checked on the host
   const FastDiv div = make_fastdiv(kbpr);
   const bool fos = p.four_over_six != 0;
   const ScaleCtx ctx = make_scale_ctx(alpha);
-  const uint32_t stride = gridDim.x * kThreads;
+  const uint32_t stride = sl.ncta * kThreads;
   auto src = [&](uint32_t b) {
     const uint32_t r = fastdiv(b, div);
     return x + (int64_t)r * q.ld + (int64_t)(b - r * kbpr) * 16;
@@ -336,10 +344,10 @@ __device__ void encode_rows(const QTensor& q, float alpha, const QBatch& p, uint
     redo_block(v, it.y, ctx, fos, codes_at(it.x), scale_at(it.x));
   };
   WarpQueue wq{qbuf, 0u};
-  uint32_t u = blockIdx.x * kThreads + threadIdx.x;
+  uint32_t u = sl.cta * kThreads + threadIdx.x;
   RawBlock<T> next;
   if (u < nblk) next.load(src(u));
-  for (uint32_t base = blockIdx.x * kThreads; base < nblk; base += stride, u += stride) {
+  for (uint32_t base = sl.cta * kThreads; base < nblk; base += stride, u += stride) {
     const RawBlock<T> cur = next;
     if (u + stride < nblk) next.load(src(u + stride));
     uint32_t st = kBlockDone, sc = 0u;
@@ -356,14 +364,15 @@ __device__ void encode_rows(const QTensor& q, float alpha, const QBatch& p, uint
     if (wq.n > kQueueCap - 32) wq.drain(redo);
   }
   wq.drain(redo);
-  if (p.sf_layout == 1) zero_sf_padding(q.scales, q.rows, kbpr);
+  if (p.sf_layout == 1) zero_sf_padding(q.scales, q.rows, kbpr, sl);
 }
 
 // Encode pass, blocks along rows; output transposed: codes [cols, rows/2],
 // scales for cols rows x rows/16 blocks.  Unit = column pair x 16 rows (two
 // blocks), the next unit's loads issued before the current one is encoded.
 template <typename T, bool RHT>
-__device__ void encode_cols(const QTensor& q, float alpha, const QBatch& p, uint2* qbuf) {
+__device__ void encode_cols(const QTensor& q, float alpha, const QBatch& p, uint2* qbuf,
+                            const Slice sl) {
   const T* x = static_cast<const T*>(q.x);
   const uint32_t ncp = (uint32_t)(q.cols >> 1);
   const uint32_t kb_total = (uint32_t)(q.rows >> 4);
@@ -372,7 +381,7 @@ __device__ void encode_cols(const QTensor& q, float alpha, const QBatch& p, uint
   const FastDiv div = make_fastdiv(ncp), div_out = make_fastdiv(kb_total);
   const bool fos = p.four_over_six != 0;
   const ScaleCtx ctx = make_scale_ctx(alpha);
-  const uint32_t stride = gridDim.x * kThreads;
+  const uint32_t stride = sl.ncta * kThreads;
   auto src = [&](uint32_t unit) {
     const uint32_t rg = fastdiv(unit, div);
     return x + (int64_t)rg * 16 * q.ld + 2 * (int64_t)(unit - rg * ncp);
@@ -388,10 +397,10 @@ __device__ void encode_cols(const QTensor& q, float alpha, const QBatch& p, uint
                q.scales + sf_offset(c, kb, kb_total, p.sf_layout));
   };
   WarpQueue wq{qbuf, 0u};
-  uint32_t u = blockIdx.x * kThreads + threadIdx.x;
+  uint32_t u = sl.cta * kThreads + threadIdx.x;
   RawPair<T> next;
   if (u < nunits) next.load(src(u), q.ld);
-  for (uint32_t base = blockIdx.x * kThreads; base < nunits; base += stride, u += stride) {
+  for (uint32_t base = sl.cta * kThreads; base < nunits; base += stride, u += stride) {
     const RawPair<T> cur = next;
     if (u + stride < nunits) next.load(src(u + stride), q.ld);
     uint32_t st[2] = {kBlockDone, kBlockDone}, sc[2] = {0u, 0u}, ob[2] = {0u, 0u};
@@ -417,7 +426,7 @@ __device__ void encode_cols(const QTensor& q, float alpha, const QBatch& p, uint
     if (wq.n > kQueueCap - 64) wq.drain(redo);
   }
   wq.drain(redo);
-  if (p.sf_layout == 1) zero_sf_padding(q.scales, q.cols, kb_total);
+  if (p.sf_layout == 1) zero_sf_padding(q.scales, q.cols, kb_total, sl);
 }
 
 // Encode pass, 16x16 tiles.  A warp holds two adjacent tiles of one 16-row
@@ -430,7 +439,8 @@ __device__ void encode_cols(const QTensor& q, float alpha, const QBatch& p, uint
 // is redone exactly by its half-warp, and rows whose codes are ambiguous are
 // queued for an exact redo under the tile's scale.
 template <typename T>
-__device__ void encode_2d(const QTensor& q, float alpha, const QBatch& p, uint2* qbuf) {
+__device__ void encode_2d(const QTensor& q, float alpha, const QBatch& p, uint2* qbuf,
+                          const Slice sl) {
   const T* x = static_cast<const T*>(q.x);
   const uint32_t kbpr = (uint32_t)(q.cols >> 4);
   const uint32_t npair = (kbpr + 1) >> 1;
@@ -456,8 +466,8 @@ __device__ void encode_2d(const QTensor& q, float alpha, const QBatch& p, uint2*
     return kb < kbpr;
   };
   WarpQueue wq{qbuf, 0u};
-  const uint32_t ustride = gridDim.x * warps;
-  uint32_t u = blockIdx.x * warps + (threadIdx.x >> 5);
+  const uint32_t ustride = sl.ncta * warps;
+  uint32_t u = sl.cta * warps + (threadIdx.x >> 5);
   // the next unit's block is loaded before the current one is encoded
   RawBlock<T> next;
   if (u < nunits) {
@@ -537,21 +547,37 @@ __device__ void encode_2d(const QTensor& q, float alpha, const QBatch& p, uint2*
     if (wq.n > kQueueCap - 32) wq.drain(redo);
   }
   wq.drain(redo);
-  if (p.sf_layout == 1) zero_sf_padding(q.scales, q.rows, kbpr);
+  if (p.sf_layout == 1) zero_sf_padding(q.scales, q.rows, kbpr, sl);
 }
 
-enum { kModeRows = 0, kModeCols = 1, kMode2D = 2 };
+// kModeMixed: 1D row-block and 2D tensors in one launch (no RHT).
+enum { kModeRows = 0, kModeCols = 1, kMode2D = 2, kModeMixed = 3 };
 
-// One CTA of the amax pass over tensor blockIdx.y: its partial maximum goes to
-// partials[t * kMaxAmaxCtas + blockIdx.x].
+// Tensor of CTA b in a mixed launch (end[] = ends of the tensors' CTA
+// ranges) and the CTA's place in that tensor's range.
+__device__ __forceinline__ int tensor_of(const int32_t* end, int n, uint32_t b, Slice& sl) {
+  int t = 0;
+  while (t < n - 1 && (int32_t)b >= end[t]) ++t;
+  const int32_t begin = t ? end[t - 1] : 0;
+  sl.cta = b - (uint32_t)begin;
+  sl.ncta = (uint32_t)(end[t] - begin);
+  return t;
+}
+
+// One CTA of the amax pass over tensor blockIdx.y (mixed: over the tensor
+// whose range holds blockIdx.x): its partial maximum goes to
+// partials[t * kMaxAmaxCtas + (its index within the tensor's CTAs)].
 template <typename T, int MODE, bool RHT>
 __global__ void __launch_bounds__(kThreads, 3) amax_kernel(const __grid_constant__ QBatch p) {
-  const int t = blockIdx.y;
+  Slice sl{blockIdx.x, gridDim.x};
+  int t = blockIdx.y;
+  if constexpr (MODE == kModeMixed) t = tensor_of(p.amax_end, p.n, blockIdx.x, sl);
   // the row-axis mode reads its input as element pairs in both passes: its
   // rows need not satisfy the contiguous path's 32-byte alignment
-  float m = MODE == kModeCols ? amax_cols<T, RHT>(p.t[t], p.mask) : amax_rows<T, RHT>(p.t[t], p.mask);
+  float m = MODE == kModeCols ? amax_cols<T, RHT>(p.t[t], p.mask, sl)
+                              : amax_rows<T, RHT>(p.t[t], p.mask, sl);
   m = block_reduce_max(m);
-  if (threadIdx.x == 0) p.partials[t * kMaxAmaxCtas + blockIdx.x] = m;
+  if (threadIdx.x == 0) p.partials[t * kMaxAmaxCtas + sl.cta] = m;
   pdl_trigger();
 }
 
@@ -568,11 +594,16 @@ __global__ void __launch_bounds__(kThreads) finalize_kernel(const __grid_constan
 // Resident CTAs per SM the encode kernels are compiled for: the row-axis mode
 // holds two 16-element columns per thread and needs the larger register file.
 template <int MODE>
-constexpr int encode_min_blocks() { return MODE == 1 ? 2 : 3; }
+constexpr int encode_min_blocks() { return MODE == kModeCols ? 2 : 3; }
 
 template <typename T, int MODE, bool RHT>
 __global__ void __launch_bounds__(kThreads, encode_min_blocks<MODE>()) encode_kernel(const __grid_constant__ QBatch p, int ga) {
-  const int t = blockIdx.y;
+  Slice sl{blockIdx.x, gridDim.x};
+  int t = blockIdx.y;
+  if constexpr (MODE == kModeMixed) {
+    t = tensor_of(p.enc_end, p.n, blockIdx.x, sl);
+    ga = p.amax_end[t] - (t ? p.amax_end[t - 1] : 0);
+  }
   float alpha;
   if (p.gs_in) {
     alpha = *p.gs_in;
@@ -580,12 +611,19 @@ __global__ void __launch_bounds__(kThreads, encode_min_blocks<MODE>()) encode_ke
     pdl_wait();
     alpha = alpha_from_amax(reduce_partials(p.partials + t * kMaxAmaxCtas, ga));
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0 && p.t[t].gs_out) *p.t[t].gs_out = alpha;
+  if (sl.cta == 0 && threadIdx.x == 0 && p.t[t].gs_out) *p.t[t].gs_out = alpha;
   __shared__ uint2 queue[kThreads / 32][kQueueCap];
   uint2* qbuf = queue[threadIdx.x >> 5];
-  if (MODE == kModeRows) encode_rows<T, RHT>(p.t[t], alpha, p, qbuf);
-  else if (MODE == kModeCols) encode_cols<T, RHT>(p.t[t], alpha, p, qbuf);
-  else encode_2d<T>(p.t[t], alpha, p, qbuf);
+  if constexpr (MODE == kModeRows) {
+    encode_rows<T, RHT>(p.t[t], alpha, p, qbuf, sl);
+  } else if constexpr (MODE == kModeCols) {
+    encode_cols<T, RHT>(p.t[t], alpha, p, qbuf, sl);
+  } else if constexpr (MODE == kMode2D) {
+    encode_2d<T>(p.t[t], alpha, p, qbuf, sl);
+  } else {
+    if (p.two_d_of[t]) encode_2d<T>(p.t[t], alpha, p, qbuf, sl);
+    else encode_rows<T, false>(p.t[t], alpha, p, qbuf, sl);
+  }
 }
 
 uint64_t max_units(const QBatch& b, int mode) {
@@ -740,7 +778,7 @@ __global__ void __launch_bounds__(kThreads)
     }
     __syncthreads();
   }
-  if (sf_out == 1) zero_sf_padding(out_scales, cols, rows >> 4);
+  if (sf_out == 1) zero_sf_padding(out_scales, cols, rows >> 4, Slice{blockIdx.x, gridDim.x});
 }
 
 // ------------------------------------------------------------------------
@@ -851,6 +889,62 @@ cudaError_t launch_typed(const QBatch& b, cudaStream_t s) {
 
 cudaError_t launch_quantize(const QBatch& b, cudaStream_t s) {
   return b.bf16 ? launch_typed<__nv_bfloat16>(b, s) : launch_typed<float>(b, s);
+}
+
+namespace {
+
+// Splits `total` CTAs between the tensors in proportion to weight[i], each
+// at least 1 and at most cap[i]; writes the ranges' ends, returns the sum.
+int32_t split_ctas(const double* weight, const uint64_t* cap, int n, uint64_t total,
+                   int32_t* end) {
+  double w = 0.0;
+  for (int i = 0; i < n; ++i) w += weight[i];
+  int32_t acc = 0;
+  for (int i = 0; i < n; ++i) {
+    uint64_t g = (uint64_t)((double)total * weight[i] / (w > 0.0 ? w : 1.0));
+    if (g > cap[i]) g = cap[i];
+    if (g < 1) g = 1;
+    acc += (int32_t)g;
+    end[i] = acc;
+  }
+  return acc;
+}
+
+template <typename T>
+cudaError_t launch_mixed_typed(QBatch& b, cudaStream_t s) {
+  double wa[kMaxBatch], we[kMaxBatch];
+  uint64_t ca[kMaxBatch], ce[kMaxBatch];
+  for (int i = 0; i < b.n; ++i) {
+    const QTensor& q = b.t[i];
+    const uint64_t blocks = (uint64_t)q.rows * (uint64_t)(q.cols / 16);
+    const uint64_t units = b.two_d_of[i] ? (uint64_t)(q.rows / 16) * (uint64_t)((q.cols / 16 + 1) / 2) * 32
+                                          : blocks;
+    wa[i] = (double)blocks;
+    // the tile encoder spends about 1.2x the row encoder's instructions per element
+    we[i] = (double)blocks * (b.two_d_of[i] ? 1.2 : 1.0);
+    ca[i] = (blocks + 4 * kThreads - 1) / (4 * kThreads);
+    if (ca[i] > (uint64_t)kMaxAmaxCtas) ca[i] = kMaxAmaxCtas;
+    ce[i] = (units + kThreads - 1) / kThreads;
+  }
+  static const int occ = [] {
+    int o = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, encode_kernel<T, kModeMixed, false>,
+                                                      kThreads, 0) != cudaSuccess ||
+        o < 1)
+      o = encode_min_blocks<kModeMixed>();
+    return o;
+  }();
+  const int32_t ga = split_ctas(wa, ca, b.n, (uint64_t)num_sms() * 3, b.amax_end);
+  const int32_t ge = split_ctas(we, ce, b.n, (uint64_t)num_sms() * (uint64_t)occ, b.enc_end);
+  cudaError_t e = launch_ex(amax_kernel<T, kModeMixed, false>, dim3(ga), s, false, b);
+  if (e != cudaSuccess) return e;
+  return launch_ex(encode_kernel<T, kModeMixed, false>, dim3(ge), s, true, b, 0);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_mixed(QBatch& b, cudaStream_t s) {
+  return b.bf16 ? launch_mixed_typed<__nv_bfloat16>(b, s) : launch_mixed_typed<float>(b, s);
 }
 
 cudaError_t launch_dequantize(const DQBatch& b, cudaStream_t s) {

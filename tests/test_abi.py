@@ -115,6 +115,32 @@ def test_batched_and_dequant_validation(lib):
     assert capi.nvfp4_dequantize(e, 1, 1, 0, None) == 1
 
 
+def test_quantize_mixed_validation(lib):
+    import ctypes
+    d = (capi.nvfp4_tensor_desc * 3)()
+    d[0] = capi.nvfp4_tensor_desc(A, None, A, A, A, 64, 128, 128)
+    d[1] = capi.nvfp4_tensor_desc(A, None, A, A, A, 40, 128, 128)  # rows % 16 != 0
+    d[2] = capi.nvfp4_tensor_desc(A, None, A, A, A, 64, 120, 120)  # cols % 16 != 0
+    flags = (ctypes.c_int32 * 3)(0, 1, 0)
+    ws = capi.nvfp4_workspace_bytes(3)
+    f = capi.nvfp4_quantize_mixed
+    # a 40-row tensor is fine in 1D, not in 16x16 tiles
+    assert f(d, flags, 2, 1, _qp(), A, ws, None) == 2
+    flags[1] = 0
+    assert f(d, flags, 3, 1, _qp(), A, ws, None) == 2   # cols % 16
+    flags[1] = 2
+    assert f(d, flags, 2, 1, _qp(), A, ws, None) == 1   # flag not 0 / 1
+    flags[1] = 1
+    d[1] = capi.nvfp4_tensor_desc(A, None, A, A, A, 64, 128, 128)
+    assert f(d, flags, 2, 1, _qp(rht_enable=1), A, ws, None) == 1
+    assert f(d, flags, 2, 1, _qp(block_axis=1), A, ws, None) == 1
+    assert f(d, flags, 2, 1, _qp(global_scale_in=A), A, ws, None) == 1
+    assert f(d, flags, 2, 1, _qp(), A, capi.nvfp4_workspace_bytes(1), None) == 4
+    assert f(d, flags, 65, 1, _qp(), A, capi.nvfp4_workspace_bytes(65), None) == 2
+    assert f(d, flags, 0, 1, _qp(), A, ws, None) == 0   # nothing to do
+    assert f(None, flags, 2, 1, _qp(), A, ws, None) == 1
+
+
 def test_rht_validation(lib):
     assert capi.nvfp4_rht16(A, 1, 64, 100, 100, 0, 0, A, None) == 2
     assert capi.nvfp4_rht16(A, 1, 60, 64, 64, 1, 0, A, None) == 2

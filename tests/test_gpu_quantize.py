@@ -159,6 +159,59 @@ def test_quantize_2d_odd_tile_count_and_fp32():
                        oracle.quantize_2d(to_oracle(w2), four_over_six=fos, sf_layout=1), "fos")
 
 
+# ------------------------------------------------------------ mixed 1D + 2D launch
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_quantize_mixed_matches_oracle(layout):
+    """1D activations (ragged rows, outlier channels, a strided view) and 2D
+    weights in one mixed call: every tensor bit-exact with the oracle's 1D /
+    2D quantization under its own global scale."""
+    x = synth.activation(21, 2, 300, 3072)
+    w = synth.weight(22, 3, 272, 3072)
+    base = synth.activation(23, 1, 130, 288, n_out=3)
+    w_small = synth.weight(24, 4, 48, 16 * 7, dtype=torch.bfloat16)  # odd tile count per band
+    xs = [x.to(DEV), w.to(DEV), base.to(DEV)[:, :208], w_small.to(DEV)]
+    flags = [False, True, False, True]
+    qs = nv.quantize_mixed(xs, flags, sf_layout=layout)
+    refs = [oracle.quantize_1d(to_oracle(x), sf_layout=layout),
+            oracle.quantize_2d(to_oracle(w), sf_layout=layout),
+            oracle.quantize_1d(to_oracle(base[:, :208]), sf_layout=layout),
+            oracle.quantize_2d(to_oracle(w_small), sf_layout=layout)]
+    for i, (q, ref) in enumerate(zip(qs, refs)):
+        assert_q_equal(q, ref, "mixed[%d]" % i)
+
+
+def test_quantize_mixed_qkv_shapes_equal_single_calls():
+    """The DiT QKV operands (X [2640, 3072] 1D, W [9216, 3072] 2D) through one
+    mixed call equal the separate quantize_1d / quantize_2d calls byte for
+    byte (those are pinned to the oracle above and at full size elsewhere),
+    and sampled rows equal the oracle directly; plus an fp32 pair and an
+    empty tensor (global scale 1, nothing else written)."""
+    x, w = synth.qkv_linear(DEV)
+    qs = nv.quantize_mixed([x, w], [False, True])
+    q1 = nv.quantize_1d(x)
+    q2 = nv.quantize_2d(w)
+    for a, b, what in ((qs[0], q1, "X"), (qs[1], q2, "W")):
+        assert torch.equal(a.codes, b.codes), what
+        assert torch.equal(a.scales, b.scales), what
+        assert torch.equal(a.alpha, b.alpha), what
+    # oracle on a band of each (alpha from the full tensor)
+    xa, wa = float(q1.alpha.cpu()[0]), float(q2.alpha.cpu()[0])
+    xr = to_oracle(x[256:384].cpu())
+    ref = oracle.quantize_1d(xr, alpha_in=xa, sf_layout=oracle.SF_ROWMAJOR)
+    assert np.array_equal(qs[0].codes[256:384].cpu().numpy(), ref[0])
+    wr = to_oracle(w[512:640].cpu())
+    ref = oracle.quantize_2d(wr, alpha_in=wa, sf_layout=oracle.SF_ROWMAJOR)
+    assert np.array_equal(qs[1].codes[512:640].cpu().numpy(), ref[0])
+    # fp32 inputs and an empty tensor in the batch
+    a32 = synth.activation(25, 1, 64, 256).float().to(DEV)
+    w32 = synth.weight(26, 1, 64, 256, dtype=torch.float32).to(DEV)
+    empty = torch.zeros(0, 256, device=DEV)
+    qs = nv.quantize_mixed([a32, empty, w32], [False, False, True])
+    assert_q_equal(qs[0], oracle.quantize_1d(to_oracle(a32.cpu()), sf_layout=1), "fp32 1d")
+    assert_q_equal(qs[2], oracle.quantize_2d(to_oracle(w32.cpu()), sf_layout=1), "fp32 2d")
+    assert float(qs[1].alpha.cpu()[0]) == 1.0
+
+
 # ------------------------------------------------------------ RHT / transposed
 def test_rht16_standalone_both_axes():
     mask = synth.rht_sign_mask(0)
