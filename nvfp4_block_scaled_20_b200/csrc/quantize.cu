@@ -85,7 +85,8 @@ struct Slice {
 
 // bf16 without the transform: the max stays on packed raw words; kAmaxDepth
 // 32-byte loads in flight per thread (enough bytes in flight per SM to cover
-// the HBM latency at two CTAs per SM).
+// the HBM latency at three CTAs per SM; the load form itself was measured not
+// to matter: non-coherent, plain, evict-first and bulk copies stream alike).
 constexpr int kAmaxDepth = 8;
 __device__ float amax_rows_bf16_raw(const QTensor& q, const Slice sl) {
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(q.x);
