@@ -78,7 +78,10 @@ typedef enum nvfp4_sf_layout {
 
 typedef enum nvfp4_epilogue {
   NVFP4_EPI_NONE = 0,
-  NVFP4_EPI_GELU_TANH = 1 /* 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))) */
+  NVFP4_EPI_GELU_TANH = 1, /* 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))) */
+  /* Or-ed into an activation: the GEMM also records the output's amax for
+   * its next quantization (see nvfp4_gemm). */
+  NVFP4_EPI_AMAX = 16
 } nvfp4_epilogue;
 
 /* Quantizer options.
@@ -100,14 +103,21 @@ typedef enum nvfp4_epilogue {
  *   sf_layout      nvfp4_sf_layout of the scale output.
  *   global_scale_in  device pointer to a_FP32; NULL => computed as
  *                  amax / (6 * 448) over the (transformed) tensor, 1.0 for an
- *                  all-zero tensor. */
+ *                  all-zero tensor.
+ *   amax_from_workspace  1: the tensor's amax is already in the workspace,
+ *                  left there by the nvfp4_gemm that produced the tensor
+ *                  (epilogue with NVFP4_EPI_AMAX, same workspace): the amax
+ *                  pass is skipped, only the encode pass runs (the fused
+ *                  "amax from the up-GEMM's epilogue" variant).  Needs
+ *                  global_scale_in NULL and rht_enable 0; ignored by
+ *                  nvfp4_global_scale.  0: the usual amax pass. */
 typedef struct nvfp4_qparams {
   int32_t four_over_six;
   int32_t rht_enable;
   uint32_t rht_sign_mask;
   int32_t block_axis;
   int32_t sf_layout;
-  int32_t reserved0;
+  int32_t amax_from_workspace;
   const float* global_scale_in;
 } nvfp4_qparams;
 
@@ -308,7 +318,14 @@ NVFP4_API nvfp4_status nvfp4_dequantize_rows(const nvfp4_tensor_desc* descs, int
  *            layout for M rows, K/16 blocks;  a_alpha device float.
  *   b_codes  device [N, K/2] (K-major),  b_sf, b_alpha likewise for N rows.
  *   out      device [M, ldo] of out_dtype (NVFP4_BF16: RNE; NVFP4_F32).
- *   epilogue nvfp4_epilogue, applied in fp32 before the conversion.
+ *   epilogue nvfp4_epilogue, applied in fp32 before the conversion;
+ *            with NVFP4_EPI_AMAX or-ed in, every CTA also writes the largest
+ *            |stored value| (after the activation and the rounding to
+ *            out_dtype; rows past M excluded) into the amax partials of ws,
+ *            which must then be nvfp4_workspace_bytes(1) bytes: a following
+ *            nvfp4_quantize_1d / _2d of out with that workspace and
+ *            qp->amax_from_workspace = 1 skips its amax pass and gives the
+ *            same codes, scales and global scale as without it.
  * Shape: M >= 1, N % 16 == 0, K % 64 == 0, ldo >= N, ldo * elem % 16 == 0.
  * Workspace: nvfp4_workspace_bytes(0) (the device error word). */
 NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf,

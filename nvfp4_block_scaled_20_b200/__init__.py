@@ -11,7 +11,8 @@ from __future__ import annotations
 from dataclasses import dataclass
 
 from . import capi
-from .capi import (NVFP4_BF16, NVFP4_EPI_GELU_TANH, NVFP4_EPI_NONE, NVFP4_F32,  # noqa: F401
+from .capi import (NVFP4_BF16, NVFP4_EPI_AMAX, NVFP4_EPI_GELU_TANH, NVFP4_EPI_NONE,  # noqa: F401
+                   NVFP4_F32,
                    NVFP4_SF_ROWMAJOR, NVFP4_SF_TCGEN05, NVFP4Error)
 
 __all__ = ["QTensor", "quantize_1d", "quantize_2d", "global_scale", "quantize_1d_batched",
@@ -62,9 +63,9 @@ def workspace(n_tensors: int = 1, device=None):
                        device=device or "cuda")
 
 
-def _qparams(four_over_six, rht, mask, block_axis, sf_layout, alpha_in):
+def _qparams(four_over_six, rht, mask, block_axis, sf_layout, alpha_in, amax_ready=False):
     return capi.nvfp4_qparams(int(four_over_six), int(rht), int(mask) & 0xFFFFFFFF,
-                              int(block_axis), int(sf_layout), 0,
+                              int(block_axis), int(sf_layout), int(bool(amax_ready)),
                               None if alpha_in is None else alpha_in.data_ptr())
 
 
@@ -78,14 +79,15 @@ def _alloc_q(rows, cols, sf_layout, device):
 
 
 def quantize_1d(x, four_over_six=True, rht=False, mask=0, block_axis=0,
-                sf_layout=NVFP4_SF_TCGEN05, alpha_in=None, ws=None, out=None, stream=None):
+                sf_layout=NVFP4_SF_TCGEN05, alpha_in=None, ws=None, out=None, stream=None,
+                amax_ready=False):
     """nvfp4_quantize_1d on a 2D CUDA tensor (row stride = x.stride(0))."""
     rows, cols = x.shape
     R, C = (rows, cols) if block_axis == 0 else (cols, rows)
     if out is None:
         out = QTensor(*_alloc_q(R, C, sf_layout, x.device), R, C, sf_layout)
     ws = workspace(1, x.device) if ws is None else ws
-    qp = _qparams(four_over_six, rht, mask, block_axis, sf_layout, alpha_in)
+    qp = _qparams(four_over_six, rht, mask, block_axis, sf_layout, alpha_in, amax_ready)
     st = capi.nvfp4_quantize_1d(x.data_ptr(), _dtype_code(x), rows, cols, x.stride(0), qp,
                                 out.codes.data_ptr(), out.scales.data_ptr(), out.alpha.data_ptr(),
                                 ws.data_ptr(), ws.numel(), _stream(stream))
@@ -239,14 +241,21 @@ def transpose_2d(q: QTensor, sf_layout=None, out=None, stream=None):
 
 
 def gemm(a: QTensor, b: QTensor, out_dtype=None, epilogue=NVFP4_EPI_NONE, out=None, ws=None,
-         stream=None):
-    """out[M, N] = a (M x K) times b (N x K) transposed, both NVFP4 (tcgen05 layout)."""
+         stream=None, amax_ws=None):
+    """out[M, N] = a (M x K) times b (N x K) transposed, both NVFP4 (tcgen05 layout).
+    amax_ws: a quantizer workspace (workspace(1)) that receives the output's
+    amax, for quantize_1d(out, ws=amax_ws, amax_ready=True); it is then the
+    GEMM's workspace too (ws must be None or the same tensor)."""
     torch = _torch()
     out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
     M, K = a.rows, a.cols
     N = b.rows
     if out is None:
         out = torch.empty((M, N), dtype=out_dtype, device=a.codes.device)
+    if amax_ws is not None:
+        if ws is not None and ws is not amax_ws:
+            raise ValueError("with amax_ws the GEMM uses that workspace")
+        ws, epilogue = amax_ws, epilogue | NVFP4_EPI_AMAX
     ws = workspace(0, a.codes.device) if ws is None else ws
     code = NVFP4_BF16 if out.dtype == torch.bfloat16 else NVFP4_F32
     st = capi.nvfp4_gemm(a.codes.data_ptr(), a.scales.data_ptr(), a.alpha.data_ptr(),

@@ -17,7 +17,7 @@ STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "ALIGN", 4: "WORKSPACE
                 6: "TIMEOUT", 7: "UNSUPPORTED"}
 NVFP4_F32, NVFP4_BF16 = 0, 1
 NVFP4_SF_ROWMAJOR, NVFP4_SF_TCGEN05 = 0, 1
-NVFP4_EPI_NONE, NVFP4_EPI_GELU_TANH = 0, 1
+NVFP4_EPI_NONE, NVFP4_EPI_GELU_TANH, NVFP4_EPI_AMAX = 0, 1, 16
 
 EXPORTED = [
     "nvfp4_workspace_bytes", "nvfp4_codes_bytes", "nvfp4_scales_bytes", "nvfp4_global_scale",
@@ -31,7 +31,7 @@ EXPORTED = [
 class nvfp4_qparams(ctypes.Structure):
     _fields_ = [("four_over_six", ctypes.c_int32), ("rht_enable", ctypes.c_int32),
                 ("rht_sign_mask", ctypes.c_uint32), ("block_axis", ctypes.c_int32),
-                ("sf_layout", ctypes.c_int32), ("reserved0", ctypes.c_int32),
+                ("sf_layout", ctypes.c_int32), ("amax_from_workspace", ctypes.c_int32),
                 ("global_scale_in", ctypes.c_void_p)]
 
 

@@ -51,6 +51,9 @@ nvfp4_status check_qparams(const nvfp4_qparams* qp, bool two_d) {
   if (qp->sf_layout != NVFP4_SF_ROWMAJOR && qp->sf_layout != NVFP4_SF_TCGEN05)
     return NVFP4_ERR_INVALID_ARG;
   if (two_d && (qp->rht_enable || qp->block_axis != 0)) return NVFP4_ERR_INVALID_ARG;
+  // a producer's amax is of the untransformed values
+  if (qp->amax_from_workspace != 0 && qp->amax_from_workspace != 1) return NVFP4_ERR_INVALID_ARG;
+  if (qp->amax_from_workspace && qp->rht_enable) return NVFP4_ERR_INVALID_ARG;
   if (qp->global_scale_in && !aligned(qp->global_scale_in, 4)) return NVFP4_ERR_ALIGN;
   return NVFP4_OK;
 }
@@ -64,6 +67,7 @@ void fill_batch_common(QBatch& b, int32_t dtype, const nvfp4_qparams* qp, void* 
   b.block_axis = qp->block_axis;
   b.sf_layout = qp->sf_layout;
   b.gs_in = qp->global_scale_in;
+  b.amax_ready = qp->amax_from_workspace != 0;
   b.partials = ws ? partials(ws) : nullptr;
   b.err = ws ? err_word(ws) : nullptr;
 }
@@ -315,13 +319,15 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
   if (!a_codes || !a_sf || !a_alpha || !b_codes || !b_sf || !b_alpha || !out)
     return NVFP4_ERR_INVALID_ARG;
   if (!dtype_ok(out_dtype)) return NVFP4_ERR_INVALID_ARG;
-  if (epilogue != NVFP4_EPI_NONE && epilogue != NVFP4_EPI_GELU_TANH) return NVFP4_ERR_INVALID_ARG;
+  const int32_t act = epilogue & ~NVFP4_EPI_AMAX;
+  if (act != NVFP4_EPI_NONE && act != NVFP4_EPI_GELU_TANH) return NVFP4_ERR_INVALID_ARG;
   if (M < 1 || N < 16 || K < 64 || N % 16 || K % 64 || ldo < N) return NVFP4_ERR_SHAPE;
   if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_sf, 16) || !aligned(b_sf, 16) ||
       !aligned(out, 16) || (ldo * elem_bytes(out_dtype)) % 16 || !aligned(a_alpha, 4) ||
       !aligned(b_alpha, 4))
     return NVFP4_ERR_ALIGN;
-  if (!ws || ws_bytes < nvfp4_workspace_bytes(0)) return NVFP4_ERR_WORKSPACE;
+  const bool want_amax = (epilogue & NVFP4_EPI_AMAX) != 0;
+  if (!ws || ws_bytes < nvfp4_workspace_bytes(want_amax ? 1 : 0)) return NVFP4_ERR_WORKSPACE;
   GemmArgs g;
   g.a_codes = a_codes;
   g.a_sf = a_sf;
@@ -337,6 +343,7 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
   g.ldo = ldo;
   g.epilogue = epilogue;
   g.err = err_word(ws);
+  g.amax_partials = want_amax ? partials(ws) : nullptr;
   bool unsupported = false;
   int e = launch_gemm(g, S(stream), &unsupported);
   if (unsupported) return NVFP4_ERR_UNSUPPORTED;

@@ -319,6 +319,11 @@ struct Params {
   int32_t out_bf16;
   int32_t epilogue;
   uint32_t* err;
+  // non-null: each CTA writes the largest |stored value| of its tiles (after
+  // the activation and the output rounding, rows past M excluded) to
+  // amax_partials[blockIdx.x]; CTA 0 zeroes the slots of absent CTAs, so a
+  // quantizer can reduce all kMaxAmaxCtas slots
+  float* amax_partials;
 };
 
 // Tile t of the grouped raster -> (tile row, tile column).
@@ -332,15 +337,25 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mt
   nt = r / gm;
 }
 
+// max(|a|, |b|) per bf16 half of two packed words (sign bits cleared).
+__device__ __forceinline__ uint32_t absmax2_bf16(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a & 0x7FFF7FFFu), "r"(b & 0x7FFF7FFFu));
+  return r;
+}
+
 // One lane's 16 accumulator columns -> x alpha_a*alpha_b, optional GELU ->
-// its row of the warp's staging chunk (32 rows x 16 columns, dense).
+// its row of the warp's staging chunk (32 rows x 16 columns, dense).  With
+// the output amax on (track) and the lane's row inside M, the largest
+// |stored value| is folded into amax (bf16 outputs: as packed bf16 pairs).
 __device__ __forceinline__ void stage16(const Params& p, uint8_t* chunk, int lane,
-                                        const uint32_t r[16], float scale) {
+                                        const uint32_t r[16], float scale, bool track,
+                                        uint32_t& amax) {
   float v[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     v[i] = __fmul_rn(__uint_as_float(r[i]), scale);
-    if (p.epilogue == 1) v[i] = gelu_tanh(v[i]);
+    if ((p.epilogue & 0xF) == 1) v[i] = gelu_tanh(v[i]);
   }
   if (p.out_bf16) {
     uint32_t w[8];
@@ -349,10 +364,20 @@ __device__ __forceinline__ void stage16(const Params& p, uint8_t* chunk, int lan
       __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
       w[i] = *reinterpret_cast<uint32_t*>(&h);
     }
+    if (track) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = absmax2_bf16(amax, w[i]);
+    }
     uint4* d4 = reinterpret_cast<uint4*>(chunk + lane * 32);
     d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
     d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
   } else {
+    if (track) {
+      float m = __uint_as_float(amax);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+      amax = __float_as_uint(m);
+    }
     float4* d4 = reinterpret_cast<float4*>(chunk + lane * 64);
 #pragma unroll
     for (int i = 0; i < 4; ++i) d4[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
@@ -381,6 +406,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   uint64_t* mma_done = ovl_free + 1;          // [1] all MMAs of the pair done (leader)
   uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  uint32_t* cta_amax = (uint32_t*)(tmem_slot + 2);  // epilogue warps' output amax
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
@@ -409,6 +435,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     mbar_init(smem_u32(ovl_free), 2 * kEpiWarps);
     mbar_init(smem_u32(mma_done), 1);
     *abort_flag = 0;
+    *cta_amax = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -533,6 +560,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const float scale = __fmul_rn(*p.a_alpha, *p.b_alpha);
     uint8_t* my_stage = sEpi + e * 2 * kEpiChunkBytes;
     uint32_t tile_i = 0, chunk_i = 0;
+    const bool want_amax = p.amax_partials != nullptr;
+    uint32_t lane_amax = 0u;  // bf16x2 pair (bf16 out) or fp32 bits (fp32 out), both >= 0
     for (int t = pair; t < num_tiles; t += num_pairs, ++tile_i) {
       const uint32_t b = tile_i & 1u, use = tile_i >> 1;
       int mt, nt;
@@ -561,7 +590,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         uint8_t* chunk = my_stage + (chunk_i & 1u) * kEpiChunkBytes;
         if (lane == 0) bulk_wait_read_one();  // this buffer's previous store has read it
         __syncwarp();
-        stage16(p, chunk, lane, r, scale);
+        stage16(p, chunk, lane, r, scale, want_amax && m0 + quad * 32 + lane < p.M, lane_amax);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -605,6 +634,20 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     // every store has left shared memory and reached global memory
     if (lane == 0) bulk_wait_all();
     __syncwarp();
+    if (want_amax) {
+      // the CTA's output amax: lanes -> warp -> the eight epilogue warps
+      const float m = p.out_bf16 ? fmaxf(__uint_as_float(lane_amax << 16),
+                                         __uint_as_float(lane_amax & 0xFFFF0000u))
+                                 : __uint_as_float(lane_amax);
+      const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(m));
+      if (lane == 0) atomicMax(cta_amax, wm);
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
+      if (e == 0 && lane == 0) {
+        p.amax_partials[blockIdx.x] = __uint_as_float(*cta_amax);
+        if (blockIdx.x == 0)
+          for (int i = gridDim.x; i < kMaxAmaxCtas; ++i) p.amax_partials[i] = 0.0f;
+      }
+    }
   } else {
     // ------------------------------------------------------------ scale staging
     // Quadrant q's lanes get, per MMA k-block k of the stage: A columns
@@ -756,6 +799,7 @@ int launch_persistent(const GemmArgs& a, cudaStream_t s) {
   p.K = (int32_t)a.K;
   p.out_bf16 = a.out_bf16;
   p.epilogue = a.epilogue;
+  p.amax_partials = a.amax_partials;
   p.err = a.err;
   // resident pairs: one pair per two SMs where the GPU's layout allows
   static const int max_pairs = [] {

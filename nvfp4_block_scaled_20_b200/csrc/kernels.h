@@ -33,6 +33,7 @@ struct QBatch {
   int32_t sf_layout;
   int32_t two_d;        // 1: 16x16 tiles (block_axis 0, no RHT)
   int32_t amax_only;    // 1: only the amax pass; writes the global scale
+  int32_t amax_ready;   // 1: the partials are already in the workspace (no amax pass)
   const float* gs_in;   // device; nullptr => from the amax pass
   float* partials;      // device, kMaxAmaxCtas slots per tensor (amax pass output)
   uint32_t* err;        // device error word
@@ -80,8 +81,9 @@ struct GemmArgs {
   void* out;
   int32_t out_bf16;
   int64_t ldo;
-  int32_t epilogue;
+  int32_t epilogue;  // activation (low 4 bits); NVFP4_EPI_AMAX bit
   uint32_t* err;  // device error word
+  float* amax_partials;  // non-null: per-CTA output amax (kMaxAmaxCtas slots)
 };
 
 int num_sms();

@@ -852,7 +852,10 @@ cudaError_t launch_mode(const QBatch& b, cudaStream_t s) {
   const uint64_t units = max_units(b, MODE);
   const uint64_t per_cta = (uint64_t)kThreads;
   int ga = 0;
-  if (!b.gs_in) {
+  if (!b.gs_in && b.amax_ready) {
+    // the producer of x left per-CTA maxima in every slot of the workspace
+    ga = kMaxAmaxCtas;
+  } else if (!b.gs_in) {
     // amax pass: three CTAs per SM (eight 32-byte loads in flight per thread)
     uint64_t want = (units + 4 * per_cta - 1) / (4 * per_cta);
     uint64_t cap = (uint64_t)num_sms() * 3;

@@ -53,7 +53,7 @@ def test_status_strings(lib):
 
 def _qp(**kw):
     d = dict(four_over_six=1, rht_enable=0, rht_sign_mask=0, block_axis=0, sf_layout=1,
-             reserved0=0, global_scale_in=None)
+             amax_from_workspace=0, global_scale_in=None)
     d.update(kw)
     return capi.nvfp4_qparams(**d)
 
@@ -139,6 +139,20 @@ def test_quantize_mixed_validation(lib):
     assert f(d, flags, 65, 1, _qp(), A, capi.nvfp4_workspace_bytes(65), None) == 2
     assert f(d, flags, 0, 1, _qp(), A, ws, None) == 0   # nothing to do
     assert f(None, flags, 2, 1, _qp(), A, ws, None) == 1
+
+
+def test_output_amax_validation(lib):
+    ws0, ws1 = capi.nvfp4_workspace_bytes(0), capi.nvfp4_workspace_bytes(1)
+    g = capi.nvfp4_gemm
+    args = lambda epi, wsb: (A, A, A, A, A, A, 64, 128, 256, A, 1, 128, epi, A, wsb, None)
+    # the output amax needs a quantizer-sized workspace for its partials
+    assert g(*args(capi.NVFP4_EPI_AMAX, ws0)) == 4
+    assert g(*args(capi.NVFP4_EPI_GELU_TANH | capi.NVFP4_EPI_AMAX, ws0)) == 4
+    assert g(*args(2 | capi.NVFP4_EPI_AMAX, ws1)) == 1       # no activation 2
+    q = capi.nvfp4_quantize_1d
+    assert q(A, 1, 64, 256, 256, _qp(amax_from_workspace=2), A, A, A, A, ws1, None) == 1
+    assert q(A, 1, 64, 256, 256, _qp(amax_from_workspace=1, rht_enable=1), A, A, A, A, ws1,
+             None) == 1
 
 
 def test_rht_validation(lib):

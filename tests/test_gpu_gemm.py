@@ -140,3 +140,27 @@ def test_dgrad_with_transposed_weight_codes(T, Nout, Kin):
         tol = gemm_tolerance(y, s, dt == torch.bfloat16)
         bad = np.argwhere(np.abs(got - y) > tol)
         assert bad.size == 0, "%d outputs out of tolerance, first %s" % (len(bad), bad[0])
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("epilogue", [nv.NVFP4_EPI_GELU_TANH, nv.NVFP4_EPI_NONE])
+def test_output_amax_feeds_the_next_quantization(out_dtype, epilogue):
+    """The GEMM records its output's amax (per CTA, in a quantizer workspace);
+    quantizing the output from that workspace without an amax pass gives the
+    same codes, scales and global scale as the usual two-pass quantization,
+    whose global scale is the oracle's; ragged M (300 rows) and N (384)."""
+    x = synth.activation(51, 1, 300, 512, device=DEV)
+    w = synth.weight(52, 1, 384, 512, device=DEV)
+    qa, qb = nv.quantize_1d(x), nv.quantize_2d(w)
+    wsq = nv.workspace(1)
+    h = nv.gemm(qa, qb, out_dtype=out_dtype, epilogue=epilogue, amax_ws=wsq)
+    fused = nv.quantize_1d(h, ws=wsq, amax_ready=True)
+    plain = nv.quantize_1d(h)
+    torch.cuda.synchronize()
+    assert nv.device_error(wsq) == 0
+    assert torch.equal(fused.alpha, plain.alpha)
+    assert torch.equal(fused.codes, plain.codes)
+    assert torch.equal(fused.scales, plain.scales)
+    ref_alpha = oracle.quantize_1d(to_oracle(h.cpu()))[2]
+    assert float(fused.alpha.cpu()[0]) == np.float32(ref_alpha)
+
