@@ -109,8 +109,11 @@ typedef enum nvfp4_epilogue {
  *                  (epilogue with NVFP4_EPI_AMAX, same workspace): the amax
  *                  pass is skipped, only the encode pass runs (the fused
  *                  "amax from the up-GEMM's epilogue" variant).  Needs
- *                  global_scale_in NULL and rht_enable 0; ignored by
- *                  nvfp4_global_scale.  0: the usual amax pass. */
+ *                  rht_enable 0 (NVFP4_ERR_INVALID_ARG otherwise) and
+ *                  global_scale_in NULL (a given scale wins); single-tensor
+ *                  quantize calls only (the batched and mixed calls return
+ *                  NVFP4_ERR_INVALID_ARG); ignored by nvfp4_global_scale.
+ *                  0: the usual amax pass. */
 typedef struct nvfp4_qparams {
   int32_t four_over_six;
   int32_t rht_enable;

@@ -123,6 +123,7 @@ nvfp4_status nvfp4_global_scale(const void* x, int32_t dtype, int64_t rows, int6
   QBatch b;
   fill_batch_common(b, dtype, qp, ws);
   b.gs_in = nullptr;
+  b.amax_ready = 0;  // this call is the amax pass
   b.amax_only = 1;
   b.n = 1;
   b.t[0] = QTensor{x, nullptr, nullptr, global_scale_out, rows, cols, ld};
@@ -152,7 +153,7 @@ nvfp4_status nvfp4_quantize_1d_batched(const nvfp4_tensor_desc* descs, int32_t n
   if (!descs || n < 0) return NVFP4_ERR_INVALID_ARG;
   nvfp4_status st = check_qparams(qp, false);
   if (st != NVFP4_OK) return st;
-  if (qp->global_scale_in) return NVFP4_ERR_INVALID_ARG;
+  if (qp->global_scale_in || qp->amax_from_workspace) return NVFP4_ERR_INVALID_ARG;
   if (!dtype_ok(dtype)) return NVFP4_ERR_INVALID_ARG;
   for (int32_t i = 0; i < n; ++i) {
     const nvfp4_tensor_desc& d = descs[i];
@@ -185,7 +186,7 @@ nvfp4_status nvfp4_quantize_mixed(const nvfp4_tensor_desc* descs, const int32_t*
   if (n > kMaxBatch) return NVFP4_ERR_SHAPE;
   nvfp4_status st = check_qparams(qp, true);  // block_axis 0, no RHT
   if (st != NVFP4_OK) return st;
-  if (qp->global_scale_in) return NVFP4_ERR_INVALID_ARG;
+  if (qp->global_scale_in || qp->amax_from_workspace) return NVFP4_ERR_INVALID_ARG;
   if (!dtype_ok(dtype)) return NVFP4_ERR_INVALID_ARG;
   for (int32_t i = 0; i < n; ++i) {
     const nvfp4_tensor_desc& d = descs[i];

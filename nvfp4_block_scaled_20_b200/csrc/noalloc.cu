@@ -53,7 +53,8 @@ extern "C" nvfp4_status nvfp4_quantize_1d_batched_noalloc(const nvfp4_tensor_des
   using namespace nvfp4;
   if (!descs || !qp || n < 0) return NVFP4_ERR_INVALID_ARG;
   if (n > kNoAllocMaxTensors) return NVFP4_ERR_SHAPE;  // more tensors than scratch slots
-  if (qp->global_scale_in || qp->block_axis != 0) return NVFP4_ERR_INVALID_ARG;
+  if (qp->global_scale_in || qp->block_axis != 0 || qp->amax_from_workspace)
+    return NVFP4_ERR_INVALID_ARG;
   if (qp->sf_layout != NVFP4_SF_ROWMAJOR && qp->sf_layout != NVFP4_SF_TCGEN05)
     return NVFP4_ERR_INVALID_ARG;
   if (dtype != NVFP4_F32 && dtype != NVFP4_BF16) return NVFP4_ERR_INVALID_ARG;

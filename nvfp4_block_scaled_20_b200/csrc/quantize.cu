@@ -852,7 +852,7 @@ cudaError_t launch_mode(const QBatch& b, cudaStream_t s) {
   const uint64_t units = max_units(b, MODE);
   const uint64_t per_cta = (uint64_t)kThreads;
   int ga = 0;
-  if (!b.gs_in && b.amax_ready) {
+  if (!b.gs_in && b.amax_ready && !b.amax_only) {
     // the producer of x left per-CTA maxima in every slot of the workspace
     ga = kMaxAmaxCtas;
   } else if (!b.gs_in) {

@@ -153,6 +153,14 @@ def test_output_amax_validation(lib):
     assert q(A, 1, 64, 256, 256, _qp(amax_from_workspace=2), A, A, A, A, ws1, None) == 1
     assert q(A, 1, 64, 256, 256, _qp(amax_from_workspace=1, rht_enable=1), A, A, A, A, ws1,
              None) == 1
+    # batched, mixed and no-workspace calls take no producer amax
+    import ctypes
+    d = (capi.nvfp4_tensor_desc * 1)()
+    d[0] = capi.nvfp4_tensor_desc(A, None, A, A, A, 64, 128, 128)
+    flags = (ctypes.c_int32 * 1)(0)
+    assert capi.nvfp4_quantize_1d_batched(d, 1, 1, _qp(amax_from_workspace=1), A, ws1, None) == 1
+    assert capi.nvfp4_quantize_mixed(d, flags, 1, 1, _qp(amax_from_workspace=1), A, ws1, None) == 1
+    assert capi.nvfp4_quantize_1d_batched_noalloc(d, 1, 1, _qp(amax_from_workspace=1), None) == 1
 
 
 def test_rht_validation(lib):
