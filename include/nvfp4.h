@@ -66,7 +66,7 @@ typedef enum nvfp4_status {
   NVFP4_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than required     */
   NVFP4_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed           */
   NVFP4_ERR_TIMEOUT = 6,     /* a bounded device wait ran out (device side) */
-  NVFP4_ERR_UNSUPPORTED = 7  /* valid request this build does not implement */
+  NVFP4_ERR_UNSUPPORTED = 7  /* valid request the library does not implement */
 } nvfp4_status;
 
 typedef enum nvfp4_dtype { NVFP4_F32 = 0, NVFP4_BF16 = 1 } nvfp4_dtype;

@@ -383,7 +383,7 @@ const char* nvfp4_status_string(int32_t s) {
     case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
     case NVFP4_ERR_CUDA: return "CUDA call failed";
     case NVFP4_ERR_TIMEOUT: return "bounded device wait timed out";
-    case NVFP4_ERR_UNSUPPORTED: return "unsupported by this build";
+    case NVFP4_ERR_UNSUPPORTED: return "not supported by this library";
     default: return "unknown status";
   }
 }

@@ -107,7 +107,7 @@ cudaError_t launch_transpose_2d(const uint8_t* codes, const uint8_t* scales, int
 cudaError_t launch_rht16(const void* x, int bf16, int64_t rows, int64_t cols, int64_t ld,
                          int block_axis, uint32_t mask, float* out, cudaStream_t s);
 // Returns 0 on success, a cudaError_t value otherwise; sets *unsupported for
-// shapes this build does not handle.
+// shapes the library does not handle.
 int launch_gemm(const GemmArgs& a, cudaStream_t s, bool* unsupported);
 
 }  // namespace nvfp4
