@@ -90,6 +90,8 @@ def lib():
         L.orc_gemm.restype = None
         L.orc_gemm.argtypes = [_U8P, _U8P, ctypes.c_float, _i32, _U8P, _U8P,
                                ctypes.c_float, _i32, _i64, _i64, _i64, _F64P, _F64P]
+        L.orc_lora_add.restype = None
+        L.orc_lora_add.argtypes = [_F32P, _F32P, _i64, _i64, _i64, ctypes.c_double, _F64P, _F64P]
         L.orc_gelu_tanh.restype = ctypes.c_double
         L.orc_gelu_tanh.argtypes = [ctypes.c_double]
         L.orc_transpose_2d.restype = _i32
@@ -137,6 +139,23 @@ def sf_offset(r: int, kb: int, kb_total: int, layout: int) -> int:
 
 def sf_bytes(rows: int, kb_total: int, layout: int) -> int:
     return lib().orc_sf_bytes(rows, kb_total, layout)
+
+
+def lora_add(y, s, u, bl, scale: float):
+    """W4A4 + LoRA: (y + scale * u bl^T, s + |scale| * sum |u bl|) for a base
+    GEMM's (y, s) [M, N], u = x A^T [M, r] and bl = B [N, r] (fp32 / widened
+    bf16).  Returns new arrays; the inputs are not modified."""
+    y = np.array(y, dtype=np.float64, copy=True, order="C")
+    s = np.array(s, dtype=np.float64, copy=True, order="C")
+    u = np.ascontiguousarray(u, dtype=np.float32)
+    bl = np.ascontiguousarray(bl, dtype=np.float32)
+    M, r = u.shape
+    N = bl.shape[0]
+    if bl.shape[1] != r or y.shape != (M, N) or s.shape != (M, N):
+        raise ValueError("shapes: y, s [M, N], u [M, r], bl [N, r]")
+    lib().orc_lora_add(_p(u, _F32P), _p(bl, _F32P), M, N, r, float(scale), _p(y, _F64P),
+                       _p(s, _F64P))
+    return y, s
 
 
 def gelu_tanh(x: float) -> float:

@@ -30,6 +30,8 @@
  *     quantization" / "Chunkwise quantization procedure".
  *   - the three GEMMs Y = X W^T etc. on NVFP4 operands: explainer §3.4, "The
  *     three GEMMs of backpropagation in NVFP4".
+ *   - the LoRA branch scale * (x A^T) B^T added to a W4A4 output: notes §3.4,
+ *     "NVFP4 training and DMD LoRA" (quantized LoRA linear).
  *
  * Where the pages leave a step open the reading taken is written next to the
  * code (global-scale formula, rounding ties, saturation, the error sum's
@@ -536,6 +538,29 @@ void orc_gemm(const uint8_t* a_codes, const uint8_t* a_sf, float a_alpha,
     }
   free(ad);
   free(bd);
+}
+
+/* Low-rank branch of a quantized LoRA linear layer (notes, §3.4 "NVFP4
+ * training and DMD LoRA": the frozen backbone's weight stays quantized and a
+ * bf16 rank-r adapter adds scale * B (A x); overview: W ~ Dequant(Q(W0)) +
+ * delta W).  Reading: the adapter's first product u = x A^T [M, r] is
+ * given (bf16 widened to fp32), the branch adds scale * u B^T to the base
+ * output.  y[m, n] += scale * sum_j u[m, j] bl[n, j] and
+ * s[m, n] += |scale| * sum_j |u[m, j] bl[n, j]| (the tolerance scale), the
+ * sum in fp64 in increasing j; y, s row-major [M, N]. */
+void orc_lora_add(const float* u, const float* bl, int64_t M, int64_t N, int64_t r,
+                  double scale, double* y, double* s) {
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t nn = 0; nn < N; ++nn) {
+      double acc = 0.0, sabs = 0.0;
+      for (int64_t j = 0; j < r; ++j) {
+        const double p = (double)u[m * r + j] * (double)bl[nn * r + j];
+        acc += p;
+        sabs += fabs(p);
+      }
+      y[m * N + nn] += scale * acc;
+      s[m * N + nn] += fabs(scale) * sabs;
+    }
 }
 
 /* GELU, tanh approximation (Hendrycks & Gimpel, 2016), in double. */
