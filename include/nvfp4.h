@@ -349,6 +349,43 @@ NVFP4_API nvfp4_status nvfp4_rht16(const void* x, int32_t dtype, int64_t rows,
                          int64_t cols, int64_t ld, int32_t block_axis,
                          uint32_t sign_mask, float* out, void* stream);
 
+/* ------------------------------------------------------------ checks ---- */
+
+/* Conformance sweep of the hardware conversions every encoder takes its
+ * rounding decisions with: the element cast to E2M1 ("rounded to the nearest
+ * E2M1 value", explainer, "Quantization rule for a tensor block") and the
+ * block-scale cast to E4M3 ("cast_E4M3 ... rounding to the nearest
+ * representable E4M3 value", same paragraph), both round-to-nearest-even and
+ * saturating (to 6 and to 448).  The encoders' bracketed decisions are exact
+ * only if both conversions are, for every fp32 input; this call lets a test
+ * compare a whole range of inputs with the formats' definitions.
+ *   target  0: out[i] = E2M1 code (sign in bit 3, low nibble) of v_i;
+ *           1: out[i] = E4M3 byte of v_i.
+ *   v_i     the fp32 value whose bit pattern is first_bits + i, 0 <= i < count;
+ *           first_bits + count <= 2^32 (NVFP4_ERR_SHAPE otherwise).
+ *   out     device, count bytes, 16-byte aligned. */
+NVFP4_API nvfp4_status nvfp4_convert_sweep(int32_t target, uint32_t first_bits, int64_t count,
+                                           uint8_t* out, void* stream);
+
+/* Bound, in nanoseconds, of every wait in nvfp4_gemm's pipeline (0 restores
+ * the default, 2 s), for the whole process, read at each nvfp4_gemm call.
+ * A wait that runs out records NVFP4_ERR_TIMEOUT in the workspace error
+ * word; the kernel then waits (with bounds of its own, independent of this
+ * one) for the copies and MMAs it issued, frees its tensor memory and
+ * returns, leaving the device usable.  The pages' system-level failure
+ * handling is outside this library; the bound is the device-side guard every
+ * kernel wait carries. */
+NVFP4_API nvfp4_status nvfp4_set_wait_limit(uint64_t ns);
+
+/* Test hook of the timeout path, for the whole process, read at each
+ * nvfp4_gemm call: with on = 1 every GEMM's MMA issuer first waits on a
+ * barrier that nothing ever completes, while the producers' first stages are
+ * in flight; the wait runs out after the nvfp4_set_wait_limit bound and the
+ * kernel takes its abort path (NVFP4_ERR_TIMEOUT in the error word, output
+ * not written).  on = 0 (the default) turns it off; other values return
+ * NVFP4_ERR_INVALID_ARG. */
+NVFP4_API nvfp4_status nvfp4_set_test_stall(int32_t on);
+
 /* ------------------------------------------------------------ status ---- */
 
 /* Synchronizes `stream`, copies the workspace's device error word to the

@@ -14,7 +14,7 @@ CSRC = os.path.join(PKG, "csrc")
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libnvfp4.so")
 OBJDIR = os.path.join(ROOT, "_build")
-SOURCES = ["quantize.cu", "gemm.cu", "api.cu", "noalloc.cu"]
+SOURCES = ["quantize.cu", "gemm.cu", "api.cu", "noalloc.cu", "selfcheck.cu"]
 HEADERS = ["device_common.cuh", "kernels.h"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -25,6 +25,7 @@ EXPORTED = [
     "nvfp4_quantize_1d_batched_noalloc", "nvfp4_dequantize", "nvfp4_dequantize_rows",
     "nvfp4_transpose_2d",
     "nvfp4_gemm", "nvfp4_rht16", "nvfp4_get_device_error", "nvfp4_status_string",
+    "nvfp4_convert_sweep", "nvfp4_set_wait_limit", "nvfp4_set_test_stall",
 ]
 
 
@@ -73,6 +74,9 @@ _SIGS = {
     "nvfp4_rht16": (_I32, [_V, _I32, _I64, _I64, _I64, _I32, _U32, _V, _V]),
     "nvfp4_get_device_error": (_I32, [_V, ctypes.POINTER(ctypes.c_int32), _V]),
     "nvfp4_status_string": (ctypes.c_char_p, [_I32]),
+    "nvfp4_convert_sweep": (_I32, [_I32, _U32, _I64, _V, _V]),
+    "nvfp4_set_wait_limit": (_I32, [ctypes.c_uint64]),
+    "nvfp4_set_test_stall": (_I32, [_I32]),
 }
 
 
@@ -172,6 +176,18 @@ def nvfp4_get_device_error(ws, stream):
     v = ctypes.c_int32(0)
     st = _call("nvfp4_get_device_error", ws, ctypes.byref(v), stream)
     return st, v.value
+
+
+def nvfp4_convert_sweep(target, first_bits, count, out, stream):
+    return _call("nvfp4_convert_sweep", target, first_bits, count, out, stream)
+
+
+def nvfp4_set_wait_limit(ns):
+    return _call("nvfp4_set_wait_limit", ns)
+
+
+def nvfp4_set_test_stall(on):
+    return _call("nvfp4_set_test_stall", on)
 
 
 def nvfp4_status_string(s):

@@ -2,6 +2,7 @@
 // validation on the host, workspace carve-up, kernel launches.  Nothing here
 // allocates device memory or synchronizes (except nvfp4_get_device_error).
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <memory>
 #include <vector>
@@ -73,6 +74,20 @@ void fill_batch_common(QBatch& b, int32_t dtype, const nvfp4_qparams* qp, void* 
 }
 
 nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+std::atomic<uint64_t> g_wait_limit_ns{0};  // 0: kDefaultWaitLimitNs
+std::atomic<int32_t> g_test_stall{0};
+
+}  // namespace
+
+uint64_t nvfp4::gemm_wait_limit_ns() {
+  const uint64_t v = g_wait_limit_ns.load();
+  return v ? v : kDefaultWaitLimitNs;
+}
+
+int32_t nvfp4::gemm_test_stall() { return g_test_stall.load(); }
+
+namespace {
 
 nvfp4_status quantize_common(const void* x, int32_t dtype, int64_t rows, int64_t cols, int64_t ld,
                              const nvfp4_qparams* qp, uint8_t* codes, uint8_t* scales,
@@ -345,6 +360,8 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
   g.epilogue = epilogue;
   g.err = err_word(ws);
   g.amax_partials = want_amax ? partials(ws) : nullptr;
+  g.wait_limit_ns = gemm_wait_limit_ns();
+  g.stall = gemm_test_stall();
   bool unsupported = false;
   int e = launch_gemm(g, S(stream), &unsupported);
   if (unsupported) return NVFP4_ERR_UNSUPPORTED;
@@ -361,6 +378,27 @@ nvfp4_status nvfp4_rht16(const void* x, int32_t dtype, int64_t rows, int64_t col
   if (rows == 0 || cols == 0) return NVFP4_OK;
   return cuda_status(launch_rht16(x, dtype == NVFP4_BF16, rows, cols, ld, block_axis, sign_mask,
                                   out, S(stream)));
+}
+
+nvfp4_status nvfp4_set_wait_limit(uint64_t ns) {
+  g_wait_limit_ns.store(ns);
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_set_test_stall(int32_t on) {
+  if (on != 0 && on != 1) return NVFP4_ERR_INVALID_ARG;
+  g_test_stall.store(on);
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_convert_sweep(int32_t target, uint32_t first_bits, int64_t count,
+                                 uint8_t* out, void* stream) {
+  if (target != 0 && target != 1) return NVFP4_ERR_INVALID_ARG;
+  if (count < 0 || (uint64_t)first_bits + (uint64_t)count > (1ull << 32)) return NVFP4_ERR_SHAPE;
+  if (count == 0) return NVFP4_OK;
+  if (!out) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(out, 16)) return NVFP4_ERR_ALIGN;
+  return cuda_status(launch_convert_sweep(target, first_bits, (uint64_t)count, out, S(stream)));
 }
 
 nvfp4_status nvfp4_get_device_error(void* ws, int32_t* error_out, void* stream) {

@@ -75,8 +75,13 @@ constexpr uint32_t kSfSlotCol = 416; // two scale slots of 48 columns
 constexpr uint32_t kSfSlotCols = 48; // A: 4 per MMA k-block (16), B: 8 per k-block (32)
 constexpr int kSfSlots = 2;
 constexpr int kGroupM = 8;           // tile raster: 8 M-tiles per group
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
-constexpr uint64_t kDrainLimitNs = 200000000ull;  // 0.2 s when draining after an abort
+// Pipeline waits give up after Params::wait_limit_ns (2 s unless the process
+// set another bound with nvfp4_set_wait_limit); the waits of the exit path --
+// copies in flight, the pair's last MMAs -- keep fixed bounds of their own, so
+// even a very short pipeline bound leaves the CTA time to let everything it
+// issued complete before it frees tensor memory and exits.
+constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s per copy in flight
+constexpr uint64_t kMmaDoneLimitNs = 2000000000ull;  // 2 s for the last MMAs
 
 // --------------------------------------------------------------- PTX wrappers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -130,6 +135,33 @@ __device__ __forceinline__ void mbar_arrive_leader(uint32_t local_bar, bool lead
                  : "memory");
   }
 }
+// Reduces the byte count a barrier's current phase still waits for
+// (accounts for copies that will never be issued).
+__device__ __forceinline__ void mbar_complete_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// Store into the leader CTA's copy of a shared-memory word, then arrive on
+// the leader's copy of a barrier with release at cluster scope (the store is
+// visible to a thread that then waits on the barrier with acquire).
+__device__ __forceinline__ void store_and_arrive_leader(uint32_t local_word, uint32_t value,
+                                                        uint32_t local_bar) {
+  uint32_t rw, rb;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(rw) : "r"(local_word));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(rb) : "r"(local_bar));
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(rw), "r"(value) : "memory");
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(rb)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2; "
+      "selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -150,6 +182,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       if (abort_flag && *abort_flag) return false;
       if (globaltimer() - t0 > limit_ns) return false;
     }
+  }
+}
+// Bounded wait with acquire at cluster scope (no abort flag).
+__device__ __forceinline__ bool mbar_wait_acq_cluster(uint32_t bar, uint32_t parity,
+                                                      uint64_t limit_ns) {
+  if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_acq_cluster(bar, parity)) return true;
+    if ((i & 63) == 0 && globaltimer() - t0 > limit_ns) return false;
   }
 }
 // Tile load into this CTA's own shared memory, completion counted on a
@@ -290,22 +332,26 @@ __host__ __device__ constexpr uint32_t instr_desc(int M, int N) {
   return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// GELU(tanh form) in fp32: 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))),
-// tanh from the hardware approximation (tanh.approx.f32, relative error about
-// 2^-11): the result is then within 0.5 |y| 2^-11 <= 2.5e-4 |y| of the exact
-// GELU of the fp32 accumulator, below the GEMM's own tolerance.
-__device__ __forceinline__ float tanh_hw(float x) {
-  float r;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
+// GELU(tanh form) in fp32: 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))).
+// tanh from the identity tanh(u) = 1 - 2 / (exp(2u) + 1), with the exp and
+// the quotient from the __expf / __fdividef intrinsics: for |2u| < 18 their
+// relative errors (a few ulp, growing with |u|) move tanh by less than 2^-18
+// absolute, and beyond it exp(2u) is either so large that the quotient
+// vanishes under the fp32 rounding of 1 - q (tanh = 1) or so small that
+// 1 - 2/(e + 1) rounds to -1; overflow to +inf gives q = 0, tanh = 1.  So
+// |GELU_gpu(y) - GELU(y)| <= 0.5 |y| 2^-18 + a few fp32 roundings of y,
+// below 2^-17 |y| -- negligible against the GEMM's 1e-3 sum_k |a_k b_k|.
+__device__ __forceinline__ float tanh_via_exp(float u) {
+  const float e = __expf(2.0f * u);
+  return 1.0f - __fdividef(2.0f, e + 1.0f);
 }
-// With fused multiply-adds: sqrt(2/pi) (y + 0.044715 y^3) = y (k0 + k0 k1 y^2)
-// and 0.5 y (1 + t) = 0.5 y t + 0.5 y (fp32 rounding, far inside the bound).
+// sqrt(2/pi) (y + 0.044715 y^3) = y (k0 + k0 k1 y^2), and 0.5 y (1 + t) =
+// 0.5 y t + 0.5 y, with fused multiply-adds (fp32 rounding only).
 __device__ __forceinline__ float gelu_tanh(float y) {
   const float k0 = 0.7978845608028654f, k01 = 0.7978845608028654f * 0.044715f;
   const float inner = y * fmaf(k01, y * y, k0);
   const float hy = 0.5f * y;
-  return fmaf(hy, tanh_hw(inner), hy);
+  return fmaf(hy, tanh_via_exp(inner), hy);
 }
 
 struct Params {
@@ -324,6 +370,8 @@ struct Params {
   // amax_partials[blockIdx.x]; CTA 0 zeroes the slots of absent CTAs, so a
   // quantizer can reduce all kMaxAmaxCtas slots
   float* amax_partials;
+  uint64_t wait_limit_ns;  // bound of each pipeline wait
+  int32_t stall;           // test hook: the MMA issuer first waits on a barrier nothing completes
 };
 
 // Tile t of the grouped raster -> (tile row, tile column).
@@ -404,9 +452,12 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   uint64_t* acc_empty = acc_full + 2;         // [2] accumulator drained by both CTAs (leader)
   uint64_t* ovl_free = acc_empty + 2;         // [1] shared columns drained by both (leader)
   uint64_t* mma_done = ovl_free + 1;          // [1] all MMAs of the pair done (leader)
-  uint32_t* tmem_slot = (uint32_t*)(mma_done + 1);
+  uint64_t* prod_end = mma_done + 1;          // [1] the peer's producer stopped (leader)
+  uint64_t* never = prod_end + 1;             // [1] nothing arrives here (timeout test hook)
+  uint32_t* tmem_slot = (uint32_t*)(never + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   uint32_t* cta_amax = (uint32_t*)(tmem_slot + 2);  // epilogue warps' output amax
+  uint32_t* peer_it = tmem_slot + 3;  // stages the peer's producer issued (leader)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
@@ -434,6 +485,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     }
     mbar_init(smem_u32(ovl_free), 2 * kEpiWarps);
     mbar_init(smem_u32(mma_done), 1);
+    mbar_init(smem_u32(prod_end), 1);
+    mbar_init(smem_u32(never), 1);
     *abort_flag = 0;
     *cta_amax = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -468,7 +521,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         for (int kt = 0; kt < num_kt; ++kt, ++it) {
           const int s = it % kStages;
           const uint32_t round = it / kStages;
-          if (!mbar_wait(smem_u32(&empty[s]), (round & 1u) ^ 1u, abort_flag, kWaitLimitNs)) {
+          if (!mbar_wait(smem_u32(&empty[s]), (round & 1u) ^ 1u, abort_flag, p.wait_limit_ns)) {
             ok = false;
             break;
           }
@@ -494,13 +547,34 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         *abort_flag = 1;
         atomicOr(p.err, kDevErrTimeout);
       }
-      // every scale load issued must have landed before the CTA retires
-      // (the codes are waited for by the leader's MMA thread) -- bounded
+      // Every copy issued must have landed before the CTA retires (bounded
+      // waits).  Stages before the last kStages issued were consumed by MMAs,
+      // so they landed.  Scale atoms complete on this CTA's own barriers.
       for (uint32_t j = (it > (uint32_t)kStages ? it - kStages : 0u); j < it; ++j)
         mbar_wait(smem_u32(&sf_in[j % kStages]), (j / kStages) & 1u, nullptr, kDrainLimitNs);
-      if (leader)
-        for (uint32_t j = (it > (uint32_t)kStages ? it - kStages : 0u); j < it; ++j)
+      // Code tiles of both CTAs complete on the leader's barriers.  After an
+      // abort the two producers may have stopped after different stage
+      // counts (at most kStages apart: a stage is reissued only after the
+      // MMAs consumed it from both CTAs), so the peer reports its count and
+      // the leader re-balances each outstanding stage's expected bytes before
+      // waiting: a stage only the peer loaded is armed for the peer's bytes, a
+      // stage only the leader loaded is credited the peer's bytes that will
+      // never come.
+      if (!leader) {
+        store_and_arrive_leader(smem_u32(peer_it), it, smem_u32(prod_end));
+      } else {
+        uint32_t it_peer = it;
+        if (mbar_wait_acq_cluster(smem_u32(prod_end), 0, p.wait_limit_ns + 5 * kDrainLimitNs))
+          it_peer = *reinterpret_cast<volatile uint32_t*>(peer_it);
+        else
+          atomicOr(p.err, kDevErrTimeout);
+        const uint32_t half = kABytes + kBBytes;
+        for (uint32_t j = it; j < it_peer; ++j) mbar_expect_tx(smem_u32(&full[j % kStages]), half);
+        for (uint32_t j = it_peer; j < it; ++j) mbar_complete_tx(smem_u32(&full[j % kStages]), half);
+        const uint32_t it_max = it > it_peer ? it : it_peer;
+        for (uint32_t j = (it_max > (uint32_t)kStages ? it_max - kStages : 0u); j < it_max; ++j)
           mbar_wait(smem_u32(&full[j % kStages]), (j / kStages) & 1u, nullptr, kDrainLimitNs);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -508,15 +582,18 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       constexpr uint32_t idesc = instr_desc(2 * BM, BN);
       uint32_t it = 0, tile_i = 0;
       bool ok = true;
+      // test hook (nvfp4_set_test_stall): a wait that runs out after the
+      // pipeline bound while the producers' first stages are in flight
+      if (p.stall && !mbar_wait(smem_u32(never), 0, abort_flag, p.wait_limit_ns)) ok = false;
       for (int t = pair; t < num_tiles && ok; t += num_pairs, ++tile_i) {
         const uint32_t b = tile_i & 1u, use = tile_i >> 1;
         // accumulator b drained by both CTAs' epilogues of tile_i - 2, and
         // the shared columns by those of tile_i - 1
-        if (use > 0 && !mbar_wait(smem_u32(&acc_empty[b]), (use - 1) & 1u, abort_flag, kWaitLimitNs)) {
+        if (use > 0 && !mbar_wait(smem_u32(&acc_empty[b]), (use - 1) & 1u, abort_flag, p.wait_limit_ns)) {
           ok = false;
           break;
         }
-        if (tile_i > 0 && !mbar_wait(smem_u32(ovl_free), (tile_i - 1) & 1u, abort_flag, kWaitLimitNs)) {
+        if (tile_i > 0 && !mbar_wait(smem_u32(ovl_free), (tile_i - 1) & 1u, abort_flag, p.wait_limit_ns)) {
           ok = false;
           break;
         }
@@ -525,8 +602,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         for (int kt = 0; kt < num_kt; ++kt, ++it) {
           const int s = it % kStages;
           const uint32_t slot = it % kSfSlots;
-          if (!mbar_wait(smem_u32(&full[s]), (it / kStages) & 1u, abort_flag, kWaitLimitNs) ||
-              !mbar_wait(smem_u32(&sf_full[slot]), (it / kSfSlots) & 1u, abort_flag, kWaitLimitNs)) {
+          if (!mbar_wait(smem_u32(&full[s]), (it / kStages) & 1u, abort_flag, p.wait_limit_ns) ||
+              !mbar_wait(smem_u32(&sf_full[slot]), (it / kSfSlots) & 1u, abort_flag, p.wait_limit_ns)) {
             ok = false;
             break;
           }
@@ -550,7 +627,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       }
       // no MMA may still run when the pair frees its tensor memory (bounded)
       tc_commit_pair(smem_u32(mma_done));
-      mbar_wait(smem_u32(mma_done), 0, nullptr, kWaitLimitNs);
+      mbar_wait(smem_u32(mma_done), 0, nullptr, kMmaDoneLimitNs);
     }
   } else if (warp < kSfWarp0) {
     // ------------------------------------------------------------ epilogue
@@ -567,7 +644,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       int mt, nt;
       tile_coords(t, num_m, num_n, mt, nt);
       const int m0 = mt * 2 * BM + (int)rank * BM, n0 = nt * BN;
-      if (!mbar_wait(smem_u32(&acc_full[b]), use & 1u, abort_flag, kWaitLimitNs)) {
+      if (!mbar_wait(smem_u32(&acc_full[b]), use & 1u, abort_flag, p.wait_limit_ns)) {
         atomicOr(p.err, kDevErrTimeout);
         *abort_flag = 1;
         break;
@@ -662,9 +739,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       for (int kt = 0; kt < num_kt; ++kt, ++it) {
         const int s = it % kStages;
         const uint32_t slot = it % kSfSlots;
-        if (!mbar_wait(smem_u32(&sf_in[s]), (it / kStages) & 1u, abort_flag, kWaitLimitNs) ||
+        if (!mbar_wait(smem_u32(&sf_in[s]), (it / kStages) & 1u, abort_flag, p.wait_limit_ns) ||
             !mbar_wait(smem_u32(&sf_empty[slot]), ((it / kSfSlots) & 1u) ^ 1u, abort_flag,
-                       kWaitLimitNs)) {
+                       p.wait_limit_ns)) {
           ok = false;
           break;
         }
@@ -801,6 +878,8 @@ int launch_persistent(const GemmArgs& a, cudaStream_t s) {
   p.epilogue = a.epilogue;
   p.amax_partials = a.amax_partials;
   p.err = a.err;
+  p.wait_limit_ns = a.wait_limit_ns;
+  p.stall = a.stall;
   // resident pairs: one pair per two SMs where the GPU's layout allows
   static const int max_pairs = [] {
     if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

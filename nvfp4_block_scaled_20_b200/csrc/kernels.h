@@ -84,7 +84,15 @@ struct GemmArgs {
   int32_t epilogue;  // activation (low 4 bits); NVFP4_EPI_AMAX bit
   uint32_t* err;  // device error word
   float* amax_partials;  // non-null: per-CTA output amax (kMaxAmaxCtas slots)
+  uint64_t wait_limit_ns;  // bound of each pipeline wait before the kernel gives up
+  int32_t stall;           // test hook (nvfp4_set_test_stall)
 };
+
+// Default bound of a GEMM pipeline wait, and the process-wide settings
+// (nvfp4_set_wait_limit, 0 restores the default; nvfp4_set_test_stall).
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+uint64_t gemm_wait_limit_ns();
+int32_t gemm_test_stall();
 
 int num_sms();
 
@@ -104,6 +112,10 @@ cudaError_t launch_dequantize_rows(const DQGather& g, cudaStream_t s);
 cudaError_t launch_transpose_2d(const uint8_t* codes, const uint8_t* scales, int sf_in,
                                 int64_t rows, int64_t cols, uint8_t* out_codes,
                                 uint8_t* out_scales, int sf_out, cudaStream_t s);
+// Hardware conversions of the fp32 bit patterns first .. first + count - 1
+// (target 0: E2M1 code per byte, 1: E4M3 byte).
+cudaError_t launch_convert_sweep(int target, uint32_t first, uint64_t count, uint8_t* out,
+                                 cudaStream_t s);
 cudaError_t launch_rht16(const void* x, int bf16, int64_t rows, int64_t cols, int64_t ld,
                          int block_axis, uint32_t mask, float* out, cudaStream_t s);
 // Returns 0 on success, a cudaError_t value otherwise; sets *unsupported for

@@ -8,7 +8,8 @@
 // tensors.  For them the per-tensor scratch of the amax pass (one partial
 // maximum per amax CTA) lives in the fixed array below, which is part of the
 // library's device image: every GPU that loads the library holds its
-// 256 + kNoAllocMaxTensors * kMaxAmaxCtas * 4 bytes (~80 KB) until exit.
+// 4 * (64 + kNoAllocMaxTensors * kMaxAmaxCtas) = 114,944 bytes (~115 KB) until
+// exit.
 #include <cstring>
 #include <mutex>
 
@@ -24,6 +25,7 @@ constexpr int kMaxDevices = 64;
 // bits) per tensor of a call.  Every slot a call reads it has written in the
 // same call, so nothing needs clearing.
 static __device__ __align__(256) uint32_t g_noalloc_amax[64 + kNoAllocMaxTensors * nvfp4::kMaxAmaxCtas];
+static_assert(sizeof(g_noalloc_amax) == 114944, "scratch size stated in the header");
 
 std::mutex g_mu;
 uint32_t* g_addr[kMaxDevices] = {};
@@ -59,12 +61,15 @@ extern "C" nvfp4_status nvfp4_quantize_1d_batched_noalloc(const nvfp4_tensor_des
     return NVFP4_ERR_INVALID_ARG;
   if (dtype != NVFP4_F32 && dtype != NVFP4_BF16) return NVFP4_ERR_INVALID_ARG;
   const int64_t esz = dtype == NVFP4_BF16 ? 2 : 4;
+  // the same per-descriptor rules as nvfp4_quantize_1d_batched, empty tensors
+  // included: an empty tensor is still launched (it receives its global
+  // scale, 1.0), so its output pointers must be valid and aligned
   for (int32_t i = 0; i < n; ++i) {
     const nvfp4_tensor_desc& d = descs[i];
     if (d.rows < 0 || d.cols < 0 || d.ld < d.cols || d.cols % 16) return NVFP4_ERR_SHAPE;
     if ((double)d.rows * (double)d.cols / 16.0 >= 4.0e9) return NVFP4_ERR_SHAPE;
-    if (d.rows == 0 || d.cols == 0) continue;
-    if (!d.x || !d.codes || !d.scales || !d.global_scale) return NVFP4_ERR_INVALID_ARG;
+    if (!d.x && d.rows > 0 && d.cols > 0) return NVFP4_ERR_INVALID_ARG;
+    if (!d.codes || !d.scales || !d.global_scale) return NVFP4_ERR_INVALID_ARG;
     if (!aligned(d.x, 32) || (d.ld * esz) % 32 || !aligned(d.codes, 16) || !aligned(d.scales, 4) ||
         !aligned(d.global_scale, 4))
       return NVFP4_ERR_ALIGN;

@@ -60,6 +60,10 @@ def lib():
         L.orc_e4m3_decode.argtypes = [_i32]
         L.orc_e4m3_encode.restype = _i32
         L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+        L.orc_e2m1_encode_bits.restype = None
+        L.orc_e2m1_encode_bits.argtypes = [_u32, _i64, _U8P]
+        L.orc_e4m3_encode_bits.restype = None
+        L.orc_e4m3_encode_bits.argtypes = [_u32, _i64, _U8P]
         L.orc_bf16_rne.restype = ctypes.c_uint16
         L.orc_bf16_rne.argtypes = [ctypes.c_float]
         L.orc_rht16_block.restype = None
@@ -123,6 +127,15 @@ def e4m3_decode(code: int) -> float:
 
 def e4m3_encode(t: float) -> int:
     return lib().orc_e4m3_encode(float(t))
+
+
+def encode_bits(target: int, first_bits: int, n: int) -> np.ndarray:
+    """The oracle's cast of every fp32 with bit pattern first_bits + i,
+    i < n: target 0 the E2M1 code, 1 the E4M3 code (uint8 each)."""
+    out = np.empty(n, dtype=np.uint8)
+    f = lib().orc_e2m1_encode_bits if target == 0 else lib().orc_e4m3_encode_bits
+    f(first_bits, n, _p(out, _U8P))
+    return out
 
 
 def bf16_rne(f: float) -> int:

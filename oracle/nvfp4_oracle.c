@@ -118,6 +118,27 @@ int orc_e4m3_encode(float t) {
   return code;
 }
 
+/* The two element/scale casts above over a contiguous range of fp32 bit
+ * patterns (first_bits + i, i < n), one code per output byte -- the oracle's
+ * side of the exhaustive conversion sweeps (no arithmetic of its own). */
+void orc_e2m1_encode_bits(uint32_t first_bits, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) {
+    uint32_t u = first_bits + (uint32_t)i;
+    float v;
+    memcpy(&v, &u, 4);
+    out[i] = (uint8_t)orc_e2m1_encode(v);
+  }
+}
+
+void orc_e4m3_encode_bits(uint32_t first_bits, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) {
+    uint32_t u = first_bits + (uint32_t)i;
+    float v;
+    memcpy(&v, &u, 4);
+    out[i] = (uint8_t)orc_e4m3_encode(v);
+  }
+}
+
 /* ------------------------------------------------------------------------ */
 /* bf16 round-to-nearest-even of an fp32 value (finite inputs)               */
 /* ------------------------------------------------------------------------ */

@@ -43,13 +43,18 @@ def assert_q_equal(q: nv.QTensor, ref, what=""):
 
 
 def gemm_tolerance(ref_y, ref_s, out_bf16: bool, gelu: bool = False):
-    """|gpu - oracle| <= 1e-3 * sum_k |a_k b_k| (+ half a bf16 ulp of the
-    reference for bf16 outputs).  With the GELU epilogue: its slope is below
-    1.13, and the hardware tanh (relative error about 2^-11) moves GELU(y) by
-    at most 0.5 |y| 2^-11 <= 2.5e-4 * sum_k |a_k b_k|."""
+    """|gpu - oracle| <= 1e-3 * S with S = sum_k |a_k b_k| (the stated GEMM
+    bound), plus half a bf16 ulp of the reference for bf16 outputs.
+
+    With the GELU epilogue the GPU applies GELU to its own accumulator y^,
+    |y^ - y| <= 1e-3 S.  GELU-tanh's slope stays below 1.13, so the exact
+    GELU of y^ is within 1.13e-3 S of the oracle's GELU(y); the epilogue's own
+    evaluation of GELU (tanh from exp) is within 2^-17 |y^| of the exact one
+    (derivation beside the device code), and |y^| <= 1.001 S, so 2^-16 S
+    covers it."""
     tol = 1e-3 * ref_s
     if gelu:
-        tol = 1.13 * tol + 2.5e-4 * ref_s + 1e-6 * np.abs(ref_y) + 1e-30
+        tol = 1.13e-3 * ref_s + 2.0 ** -16 * ref_s
     if out_bf16:
         mag = np.abs(ref_y)
         e = np.floor(np.log2(np.where(mag > 0, mag, 1e-300)))

@@ -164,3 +164,37 @@ def test_output_amax_feeds_the_next_quantization(out_dtype, epilogue):
     ref_alpha = oracle.quantize_1d(to_oracle(h.cpu()))[2]
     assert float(fused.alpha.cpu()[0]) == np.float32(ref_alpha)
 
+
+
+def test_gelu_epilogue_on_exact_products():
+    """The epilogue's GELU evaluation alone: with K = 64 and one nonzero
+    element per row (E2M1 value times its E4M3 block scale), every output is
+    a single product y that the fp32 accumulator holds exactly, swept over
+    [-8, 8] (all 16 codes x 8 A scales x 16 B scales).  The fp32 output must
+    be within 2^-17 |y| (the evaluation bound stated beside the device code)
+    plus its own fp32 rounding of the oracle's double GELU-tanh of y."""
+    M, N, K = 128, 256, 64
+    kb = K // 16
+    a_codes = np.zeros((M, K // 2), np.uint8)
+    b_codes = np.zeros((N, K // 2), np.uint8)
+    a_codes[:, 0] = np.arange(M) % 16
+    b_codes[:, 0] = np.arange(N) % 16
+    ea = (0x30 + (np.arange(M) // 16) % 8).astype(np.uint8)   # 0.5 .. 0.9375
+    eb = (0x28 + (np.arange(N) // 16) % 16).astype(np.uint8)  # 0.25 .. 0.9375
+    a_sf = np.zeros(oracle.sf_bytes(M, kb, oracle.SF_TCGEN05), np.uint8)
+    b_sf = np.zeros(oracle.sf_bytes(N, kb, oracle.SF_TCGEN05), np.uint8)
+    for r in range(M):
+        a_sf[oracle.sf_offset(r, 0, kb, oracle.SF_TCGEN05)] = ea[r]
+    for r in range(N):
+        b_sf[oracle.sf_offset(r, 0, kb, oracle.SF_TCGEN05)] = eb[r]
+    aref, bref = (a_codes, a_sf, 1.0), (b_codes, b_sf, 0.25)
+    y, s = oracle_gemm_ref(aref, bref, M, N, K)
+    assert np.array_equal(np.abs(y), s) and np.abs(y).max() <= 8.0 and len(np.unique(y)) > 300
+    out = nv.gemm(upload(aref, M, K), upload(bref, N, K), out_dtype=torch.float32,
+                  epilogue=nv.NVFP4_EPI_GELU_TANH)
+    got = out.cpu().numpy().astype(np.float64)
+    want = np.vectorize(oracle.gelu_tanh)(y)
+    tol = 2.0 ** -17 * np.abs(y) + 2.0 ** -23 * np.abs(want)
+    bad = np.argwhere(np.abs(got - want) > tol)
+    assert bad.size == 0, "%d outputs, first y=%r gpu=%r ref=%r" % (
+        len(bad), y[tuple(bad[0])], got[tuple(bad[0])], want[tuple(bad[0])])

@@ -169,3 +169,19 @@ def test_bf16_rne_matches_torch(orc):
     want = torch.from_numpy(xs).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
     got = np.array([orc.bf16_rne(float(x)) for x in xs], dtype=np.uint16)
     assert np.array_equal(got, want)
+
+
+# ------------------------------------------------------------------ range casts
+def test_range_casts_equal_the_scalar_casts(orc):
+    """encode_bits (the oracle's side of the GPU conversion sweeps) is the
+    scalar casts applied to consecutive bit patterns: checked on ranges that
+    hold every E2M1 tie, the E4M3 saturation point and signed zeros."""
+    for target, first, n in ((0, 0x3E000000, 4096), (0, 0x40A00000 - 2048, 4096),
+                             (0, 0x7FFFF000, 8192), (1, 0x43DFF000, 8192),
+                             (1, 0x3A000000 - 100, 200), (1, 0x7F7FFFF0, 17)):
+        got = orc.encode_bits(target, first, n)
+        bits = (np.arange(n, dtype=np.uint64) + first).astype(np.uint32)
+        vals = bits.view(np.float32)
+        f = orc.e2m1_encode if target == 0 else orc.e4m3_encode
+        want = np.array([f(float(v)) if np.isfinite(v) else f(float(v)) for v in vals], np.uint8)
+        assert np.array_equal(got, want), (target, hex(first))

@@ -140,6 +140,35 @@ def test_gemm_single_block_is_scalar_product(orc):
     assert s[0, 0] == 0.5 * 3.0 * 1.0 * 2.25 * sum(abs(val(int(a)) * val(int(b))) for a, b in zip(qa, qb))
 
 
+def _gelu_tanh_decimal(x: float) -> float:
+    """0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) at 50 significant
+    digits with the decimal module: pi from its digits, the square root and
+    the exponential from decimal's own correctly rounded routines, tanh from
+    the identity tanh(u) = (e^(2u) - 1) / (e^(2u) + 1).  Independent of the
+    C library the oracle calls."""
+    from decimal import Decimal, getcontext
+    getcontext().prec = 50
+    pi = Decimal("3.14159265358979323846264338327950288419716939937510")
+    X = Decimal(x)
+    u = (Decimal(2) / pi).sqrt() * (X + Decimal("0.044715") * X * X * X)
+    e = (2 * u).exp()
+    return float(Decimal("0.5") * X * (1 + (e - 1) / (e + 1)))
+
+
+def test_gelu_tanh_against_an_independent_evaluation(orc):
+    """The tanh-form GELU at points spanning its curved range and tails,
+    within a few double ulps of max(|GELU(x)|, |x|) of the 50-digit
+    evaluation (in the negative tail 1 + tanh(u) cancels, so the double
+    formula is accurate to |x| ulps there, not to GELU's own): a coefficient
+    off in its fourth digit, a dropped cubic term or a sign error fails by
+    orders of magnitude more."""
+    for x in [-8.0, -5.5, -3.0, -2.25, -1.0, -0.5, -0.125, 1e-6, 0.25, 0.7, 1.0, 1.5, 2.0,
+              3.25, 4.5, 7.0]:
+        want = _gelu_tanh_decimal(x)
+        got = orc.gelu_tanh(x)
+        assert abs(got - want) <= 4e-16 * max(abs(want), abs(x)), (x, got, want)
+
+
 def test_gelu_tanh(orc):
     assert orc.gelu_tanh(0.0) == 0.0
     for x in np.linspace(-6, 6, 61):
