@@ -91,6 +91,21 @@ def normal(seed: int, sid: int, n: int, device="cpu") -> torch.Tensor:
     return out
 
 
+def normal_at(seed: int, sid: int, idx: torch.Tensor) -> torch.Tensor:
+    """normal(seed, sid, n)[idx] for an index tensor, without drawing the rest:
+    element i is one half of the Box-Muller pair i // 2 (uniforms 2 (i // 2)
+    and 2 (i // 2) + 1 of the stream)."""
+    key = _s64(stream_key(seed, sid))
+    pair = idx // 2
+    r1 = _mix64((2 * pair) * _s64(GAMMA) + key)
+    r2 = _mix64((2 * pair + 1) * _s64(GAMMA) + key)
+    u1 = (_lsr(r1, 11).to(torch.float64) + 0.5) * (2.0 ** -53)
+    u2 = (_lsr(r2, 11).to(torch.float64) + 0.5) * (2.0 ** -53)
+    rad = torch.sqrt(-2.0 * torch.log(u1))
+    ang = (2.0 * math.pi) * u2
+    return torch.where(idx % 2 == 0, rad * torch.cos(ang), rad * torch.sin(ang))
+
+
 def student_t3(seed: int, sid: int, n: int, device="cpu") -> torch.Tensor:
     z0 = normal(seed, sid * 4 + 0x10000, n, device)
     chi = normal(seed, sid * 4 + 0x10001, n, device) ** 2
@@ -144,6 +159,26 @@ def activation(seed: int, sid: int, rows: int, cols: int, dtype=torch.bfloat16,
             t = student_t3(seed, sid, rows * n_out, device).reshape(rows, n_out)
             x[:, cols_sel] = t * factor
     return _finish(x.reshape(-1), rows, cols, dtype)
+
+
+def activation_cols(seed: int, sid: int, rows: int, cols: int, c0: int, c1: int,
+                    dtype=torch.bfloat16, n_out: int | None = None, factor: float = 8.0,
+                    std: float = 1.0) -> torch.Tensor:
+    """activation(seed, sid, rows, cols, ...)[:, c0:c1] (mode "student_t"),
+    drawn on the host without the other columns."""
+    r = torch.arange(rows, dtype=torch.int64)[:, None]
+    c = torch.arange(c0, c1, dtype=torch.int64)[None, :]
+    x = normal_at(seed, sid, (r * cols + c).reshape(-1)).reshape(rows, c1 - c0) * std
+    if n_out is None:
+        n_out = math.ceil(0.01 * cols)
+    if n_out > 0:
+        sel = choose_columns(seed, sid + 0x5000, cols, n_out)
+        hit = [(j, col) for j, col in enumerate(sel) if c0 <= col < c1]
+        if hit:
+            t = student_t3(seed, sid, rows * n_out).reshape(rows, n_out)
+            for j, col in hit:
+                x[:, col - c0] = t[:, j] * factor
+    return _finish(x.reshape(-1), rows, c1 - c0, dtype)
 
 
 def kv_tensor(seed: int, layer: int, which: int, heads: int = 24, tokens: int = 32760,

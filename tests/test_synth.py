@@ -68,3 +68,14 @@ def test_kv_recipe_bias_per_head():
     means = kv.float().reshape(4, -1).mean(dim=1)
     bias = synth.normal(3, 0x100 + 0x8000, 4) * 2.0
     assert torch.allclose(means.double(), bias, atol=0.05)
+
+
+def test_activation_cols_is_a_column_slice_of_activation():
+    from nvfp4_block_scaled_20_b200 import synth
+    full = synth.activation(4, 2, 96, 1440)  # 15 outlier columns
+    for c0, c1 in ((0, 64), (96, 352), (1376, 1440)):
+        part = synth.activation_cols(4, 2, 96, 1440, c0, c1)
+        assert torch.equal(part, full[:, c0:c1]), (c0, c1)
+    full = synth.activation(4, 1, 64, 320, n_out=0, std=1e-3)
+    assert torch.equal(synth.activation_cols(4, 1, 64, 320, 32, 96, n_out=0, std=1e-3),
+                       full[:, 32:96])
