@@ -145,23 +145,38 @@ __device__ __forceinline__ uint64_t e2m1x2_to_f32x2(uint32_t byte) {
 // ----------------------------------------------------------------- RHT
 // y = 1/4 * H16 * diag(s) * x, s_j = -1 where bit j of mask is set.  Sign
 // flip, butterflies with strides 1, 2, 4, 8 ((a, b) -> (a + b, a - b), fp32
-// RN), then the exact scaling by 1/4.
+// RN), then the exact scaling by 1/4.  Strides 2, 4 and 8 pair elements of
+// equal parity, so they run on packed pairs (v[2k], v[2k+1]): each lane of a
+// packed add is the same IEEE operation as the scalar one.
+__device__ __forceinline__ void rht16_butterflies(float v[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    const float a = v[i], b = v[i + 1];
+    v[i] = __fadd_rn(a, b);
+    v[i + 1] = __fsub_rn(a, b);
+  }
+  uint64_t P[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) P[k] = pack2(v[2 * k], v[2 * k + 1]);
+#pragma unroll
+  for (int hp = 1; hp < 8; hp <<= 1) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (k & hp) continue;
+      const uint64_t a = P[k], b = P[k + hp];
+      P[k] = add2(a, b);
+      P[k + hp] = sub2(a, b);
+    }
+  }
+  const uint64_t quarter = pack2(0.25f, 0.25f);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) unpack2(mul2(P[k], quarter), v[2 * k], v[2 * k + 1]);
+}
 __device__ __forceinline__ void rht16(float v[16], uint32_t mask) {
 #pragma unroll
   for (int j = 0; j < 16; ++j)
     v[j] = __uint_as_float(__float_as_uint(v[j]) ^ (((mask >> j) & 1u) << 31));
-#pragma unroll
-  for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if (i & h) continue;
-      float a = v[i], b = v[i + h];
-      v[i] = __fadd_rn(a, b);
-      v[i + h] = __fsub_rn(a, b);
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], 0.25f);
+  rht16_butterflies(v);
 }
 
 // ----------------------------------------------------------------- encoder
@@ -557,6 +572,141 @@ __device__ __forceinline__ uint32_t quantize_block16_try(const float y[16], cons
   if (!rcp_ok(sw)) return kBlockCodes;
   uint32_t w[2];
   const bool ok = codes16_try(y, rcp_approx(sw), w);
+  lo = w[0];
+  hi = w[1];
+  return ok ? kBlockDone : kBlockCodes;
+}
+
+// ----------------------------------------------------------------- packed encoder
+// The block encoder above, on a block held as 8 packed fp32 pairs (element 2k
+// in the low half of yy[k]) from its first step to its last, so no pair is
+// ever re-packed; both candidate scale codes are bracketed and decoded as one
+// pair.  Every result it reports as final equals quantize_block16's (same
+// arithmetic, same certified bounds); the rest it hands back.
+
+// Raw bf16 words of a block -> packed fp32 pairs (exact).
+__device__ __forceinline__ void widen_pairs(const uint32_t w[8], uint64_t yy[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    yy[k] = pack2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xFFFF0000u));
+}
+__device__ __forceinline__ void pairs_of(const float v[16], uint64_t yy[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) yy[k] = pack2(v[2 * k], v[2 * k + 1]);
+}
+
+// max |y| over the 16 bf16 values of a raw block (an exact selection): per
+// half, max.xorsign.abs keeps max(|a|, |b|) as the magnitude.
+__device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ float absmax16_raw(const uint32_t w[8]) {
+  const uint32_t a = maxabs_bf16x2(maxabs_bf16x2(w[0], w[1]), maxabs_bf16x2(w[2], w[3]));
+  const uint32_t b = maxabs_bf16x2(maxabs_bf16x2(w[4], w[5]), maxabs_bf16x2(w[6], w[7]));
+  const uint32_t m = maxabs_bf16x2(a, b) & 0x7FFF7FFFu;
+  return fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xFFFF0000u));
+}
+__device__ __forceinline__ float absmax16_pairs(const uint64_t yy[8]) {
+  float m = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float a, b;
+    unpack2(yy[k], a, b);
+    m = fmaxf(m, fmaxf(fabsf(a), fabsf(b)));
+  }
+  return m;
+}
+
+// Both candidate scale codes from one bracket pair: t = (t6, t4) =
+// bmax * (c6, c4) (the same products as scale_codes_try), bracketed by
+// (1 +- 2^-20); false when either code is ambiguous.  *pair: the 6-code in
+// bits 0-7, the 4-code in bits 8-15.
+__device__ __forceinline__ bool scale_pair_try(float bmax, const ScaleCtx& c, uint32_t& pair) {
+  if (!c.fast) return false;
+  const uint64_t t = mul2(pack2(bmax, bmax), pack2(c.c6, c.c4));
+  float t6u, t4u, t6d, t4d;
+  unpack2(mul2(t, pack2(kUp, kUp)), t6u, t4u);
+  unpack2(mul2(t, pack2(kDn, kDn)), t6d, t4d);
+  const uint32_t pu = f32x2_to_e4m3x2(t4u, t6u), pd = f32x2_to_e4m3x2(t4d, t6d);
+  pair = pu & 0xFFFFu;
+  return (pu & 0xFFFFu) == (pd & 0xFFFFu);
+}
+
+// (s6, s4) = (dec(e6) * alpha, dec(e4) * alpha) for a code pair as above.
+__device__ __forceinline__ uint64_t scale_pair_values(uint32_t pair, float alpha) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)pair));
+  const float d6 = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+  const float d4 = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+  return mul2(pack2(d6, d4), pack2(alpha, alpha));
+}
+
+// approx_err16 on packed pairs.
+__device__ __forceinline__ float approx_err16_pairs(const uint64_t yy[8], float r) {
+  const uint64_t rr = pack2(r, r);
+  uint64_t acc[2] = {0ull, 0ull};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint64_t q = mul2(yy[k], rr);
+    const uint64_t d = sub2(q, e2m1_round_pair(q));
+    acc[k & 1] = fma2(d, d, acc[k & 1]);
+  }
+  float a0, a1;
+  unpack2(add2(acc[0], acc[1]), a0, a1);
+  return a0 + a1;
+}
+
+// codes16_try on packed pairs.
+__device__ __forceinline__ bool codes16_try_pairs(const uint64_t yy[8], float r, uint32_t w[2]) {
+  const float ru = r * kUp, rd = r * kDn;
+  const uint64_t up = pack2(ru, ru), dn = pack2(rd, rd);
+  uint32_t diff = 0u;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float a[8], b[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      unpack2(mul2(yy[4 * h + k], up), a[2 * k], a[2 * k + 1]);
+      unpack2(mul2(yy[4 * h + k], dn), b[2 * k], b[2 * k + 1]);
+    }
+    w[h] = cvt8_e2m1(a);
+    diff |= w[h] ^ cvt8_e2m1(b);
+  }
+  return diff == 0u;
+}
+
+// quantize_block16_try on packed pairs with the block max given.
+__device__ __forceinline__ uint32_t quantize_block16_pairs(const uint64_t yy[8], float bmax,
+                                                           const ScaleCtx& ctx, bool four_over_six,
+                                                           uint32_t& lo, uint32_t& hi,
+                                                           uint32_t& scale) {
+  uint32_t pair;
+  if (!scale_pair_try(bmax, ctx, pair)) return kBlockExact;
+  const uint32_t e6 = pair & 0xFFu, e4 = pair >> 8;
+  float s6, s4;
+  unpack2(scale_pair_values(pair, ctx.alpha), s6, s4);
+  uint32_t ew = e6;
+  float sw = s6;
+  if (four_over_six && e4 != e6) {  // equal codes: identical candidates, 6 wins the tie
+    if (!fast_pick_ok(e6, s6, s4)) return kBlockExact;
+    const int pick = certified_pick(approx_err16_pairs(yy, rcp_approx(s6)), s6,
+                                    approx_err16_pairs(yy, rcp_approx(s4)), s4, kPickMargin);
+    if (pick == 2) return kBlockExact;
+    if (pick == 1) {
+      ew = e4;
+      sw = s4;
+    }
+  }
+  scale = ew;
+  if (sw == 0.0f) {
+    lo = hi = 0u;
+    return kBlockDone;
+  }
+  if (!rcp_ok(sw)) return kBlockCodes;
+  uint32_t w[2];
+  const bool ok = codes16_try_pairs(yy, rcp_approx(sw), w);
   lo = w[0];
   hi = w[1];
   return ok ? kBlockDone : kBlockCodes;

@@ -796,18 +796,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (EncodeTiledFn)ptr;
-  }
-  return fn;
-}
+EncodeTiledFn encode_fn() { return (EncodeTiledFn)tensor_map_encoder(); }
 
 // Codes [rows, K/2] bytes, box = 128 bytes x box_rows rows, 128-byte swizzle,
 // out-of-bounds rows / columns read as zero.
@@ -901,6 +890,19 @@ int launch_persistent(const GemmArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+void* tensor_map_encoder() {
+  static void* fn = [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      ptr = nullptr;
+    return ptr;
+  }();
+  return fn;
+}
 
 int launch_gemm(const GemmArgs& a, cudaStream_t s, bool* unsupported) {
   *unsupported = false;

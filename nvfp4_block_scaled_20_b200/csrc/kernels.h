@@ -95,6 +95,8 @@ uint64_t gemm_wait_limit_ns();
 int32_t gemm_test_stall();
 
 int num_sms();
+// The driver's cuTensorMapEncodeTiled (looked up once), or nullptr.
+void* tensor_map_encoder();
 
 // Each returns a cudaError_t from the launch.
 // Quantization: an amax kernel writing per-CTA partial maxima, then the

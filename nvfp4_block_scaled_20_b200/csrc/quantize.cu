@@ -13,6 +13,8 @@
 // A tensor that fits in L2 is read from HBM once: the encode pass finds it in
 // L2.  Batched calls (KV cache) carry up to kMaxBatch tensors in the kernel
 // parameters, one tensor per blockIdx.y.
+#include <cuda.h>
+
 #include <type_traits>
 
 #include "device_common.cuh"
@@ -256,6 +258,20 @@ template <> struct RawBlock<__nv_bfloat16> {
       v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
   }
+  // the block as packed fp32 pairs (after the transform when RHT) and its max |y|
+  template <bool RHT>
+  __device__ __forceinline__ float prepare(uint64_t yy[8], uint32_t mask) const {
+    if constexpr (RHT) {
+      float v[16];
+      widen(v);
+      rht16(v, mask);
+      pairs_of(v, yy);
+      return absmax16(v);
+    } else {
+      widen_pairs(w, yy);
+      return absmax16_raw(w);
+    }
+  }
 };
 template <> struct RawBlock<float> {
   float f[16];
@@ -263,6 +279,14 @@ template <> struct RawBlock<float> {
   __device__ __forceinline__ void widen(float v[16]) const {
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = f[i];
+  }
+  template <bool RHT>
+  __device__ __forceinline__ float prepare(uint64_t yy[8], uint32_t mask) const {
+    float v[16];
+    widen(v);
+    if (RHT) rht16(v, mask);
+    pairs_of(v, yy);
+    return absmax16(v);
   }
 };
 
@@ -276,15 +300,25 @@ constexpr uint32_t kRedoAll = 0xFFFFFFFFu;  // redo the pick as well
 struct WarpQueue {
   uint2* item;  // shared memory, kQueueCap entries
   uint32_t n;   // same value on every lane
-  __device__ __forceinline__ void push(bool need, uint32_t idx, uint32_t code) {
+  uint4* data;  // shared memory, 2 x 16 bytes per entry (the block's raw input), or nullptr
+  __device__ __forceinline__ void push(bool need, uint32_t idx, uint32_t code,
+                                       const uint32_t* raw8 = nullptr) {
     const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
-    if (need) item[n + __popc(m & ((1u << (threadIdx.x & 31)) - 1u))] = make_uint2(idx, code);
+    if (need) {
+      const uint32_t slot = n + __popc(m & ((1u << (threadIdx.x & 31)) - 1u));
+      item[slot] = make_uint2(idx, code);
+      if (raw8) {
+        data[2 * slot] = make_uint4(raw8[0], raw8[1], raw8[2], raw8[3]);
+        data[2 * slot + 1] = make_uint4(raw8[4], raw8[5], raw8[6], raw8[7]);
+      }
+    }
     n += __popc(m);
   }
+  // redo(entry, its 32 raw bytes or garbage when pushed without them)
   template <typename F>
   __device__ __forceinline__ void drain(F&& redo) {
     __syncwarp();
-    for (uint32_t i = threadIdx.x & 31; i < n; i += 32) redo(item[i]);
+    for (uint32_t i = threadIdx.x & 31; i < n; i += 32) redo(item[i], data + 2 * i);
     __syncwarp();
     n = 0;
   }
@@ -316,7 +350,7 @@ __device__ __forceinline__ void redo_block(const float v[16], uint32_t code, con
 // encoded.
 template <typename T, bool RHT>
 __device__ void encode_rows(const QTensor& q, float alpha, const QBatch& p, uint2* qbuf,
-                            const Slice sl) {
+                            uint4* qdata, const Slice sl) {
   const T* x = static_cast<const T*>(q.x);
   const uint32_t kbpr = (uint32_t)(q.cols >> 4);
   const uint32_t nblk = (uint32_t)q.rows * kbpr;  // < 2^32, checked on the host
@@ -336,15 +370,27 @@ __device__ void encode_rows(const QTensor& q, float alpha, const QBatch& p, uint
     const uint32_t r = fastdiv(b, div);
     return q.scales + sf_offset(r, b - r * kbpr, kbpr, p.sf_layout);
   };
-  auto redo = [&](uint2 it) {
-    RawBlock<T> blk;
-    blk.load(src(it.x));
+  // bf16 blocks are queued with their raw input, fp32 blocks are reloaded
+  constexpr bool kCarry = std::is_same<T, __nv_bfloat16>::value;
+  auto redo = [&](uint2 it, const uint4* d) {
     float v[16];
-    blk.widen(v);
+    if constexpr (kCarry) {
+      const uint4 d0 = d[0], d1 = d[1];
+      const uint32_t w[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+    } else {
+      RawBlock<T> blk;
+      blk.load(src(it.x));
+      blk.widen(v);
+    }
     if (RHT) rht16(v, p.mask);
     redo_block(v, it.y, ctx, fos, codes_at(it.x), scale_at(it.x));
   };
-  WarpQueue wq{qbuf, 0u};
+  WarpQueue wq{qbuf, 0u, qdata};
   uint32_t u = sl.cta * kThreads + threadIdx.x;
   RawBlock<T> next;
   if (u < nblk) next.load(src(u));
@@ -353,15 +399,24 @@ __device__ void encode_rows(const QTensor& q, float alpha, const QBatch& p, uint
     if (u + stride < nblk) next.load(src(u + stride));
     uint32_t st = kBlockDone, sc = 0u;
     if (u < nblk) {
+      uint32_t lo, hi;
+#if NVFP4_ROWS_PACKED
+      uint64_t yy[8];
+      const float bmax = cur.template prepare<RHT>(yy, p.mask);
+      st = quantize_block16_pairs(yy, bmax, ctx, fos, lo, hi, sc);
+#else
       float v[16];
       cur.widen(v);
       if (RHT) rht16(v, p.mask);
-      uint32_t lo, hi;
       st = quantize_block16_try(v, ctx, fos, lo, hi, sc);
+#endif
       if (st == kBlockDone) store_codes(codes_at(u), lo, hi);
       if (st != kBlockExact) *scale_at(u) = (uint8_t)sc;
     }
-    wq.push(st != kBlockDone, u, st == kBlockExact ? kRedoAll : sc);
+    if constexpr (kCarry)
+      wq.push(st != kBlockDone, u, st == kBlockExact ? kRedoAll : sc, cur.w);
+    else
+      wq.push(st != kBlockDone, u, st == kBlockExact ? kRedoAll : sc);
     if (wq.n > kQueueCap - 32) wq.drain(redo);
   }
   wq.drain(redo);
@@ -388,7 +443,7 @@ __device__ void encode_cols(const QTensor& q, float alpha, const QBatch& p, uint
     return x + (int64_t)rg * 16 * q.ld + 2 * (int64_t)(unit - rg * ncp);
   };
   // queued entries hold the output block index c * kb_total + kb
-  auto redo = [&](uint2 it) {
+  auto redo = [&](uint2 it, const uint4*) {
     const uint32_t c = fastdiv(it.x, div_out), kb = it.x - c * kb_total;
     float v[16];
 #pragma unroll
@@ -397,7 +452,7 @@ __device__ void encode_cols(const QTensor& q, float alpha, const QBatch& p, uint
     redo_block(v, it.y, ctx, fos, q.codes + (int64_t)c * out_row_bytes + (int64_t)kb * 8,
                q.scales + sf_offset(c, kb, kb_total, p.sf_layout));
   };
-  WarpQueue wq{qbuf, 0u};
+  WarpQueue wq{qbuf, 0u, nullptr};
   uint32_t u = sl.cta * kThreads + threadIdx.x;
   RawPair<T> next;
   if (u < nunits) next.load(src(u), q.ld);
@@ -430,6 +485,250 @@ __device__ void encode_cols(const QTensor& q, float alpha, const QBatch& p, uint
   if (p.sf_layout == 1) zero_sf_padding(q.scales, q.cols, kb_total, sl);
 }
 
+// ------------------------------------------------------------------------
+// Row-axis (transposing) mode for bf16 inputs, staged through shared memory
+// by TMA.  The input is walked in tiles of 64 rows x 128 columns (16 KB, one
+// cp.async.bulk.tensor each, zero-filled past the tensor's edges), kTmaStages
+// tiles in flight per CTA.  In a tile, thread t owns the column pair
+// 2 (t % 64), 2 (t % 64) + 1 and the 16-row group t / 64: it reads its 16
+// words (one bf16 pair per row) from shared memory -- a warp reads 32
+// consecutive words of a row, conflict-free -- and handles the two
+// 16-element blocks along rows; the four row groups of a tile fill one
+// 32-byte run of each output row's codes.  A bounded wait that runs out
+// records NVFP4_ERR_TIMEOUT; the CTA then waits for its loads in flight
+// (bounded) and stops.
+constexpr int kTmaRows = 64, kTmaCols = 128;
+constexpr int kTmaTileBytes = kTmaRows * kTmaCols * 2;
+constexpr int kTmaStages = 4;
+constexpr int kTmaSmemBytes = kTmaStages * kTmaTileBytes + 128;
+constexpr uint64_t kTmaWaitNs = 2000000000ull, kTmaDrainNs = 200000000ull;
+
+struct ColsMaps {
+  CUtensorMap m[kMaxBatch];
+};
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ bool bar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  if (bar_try(bar, parity)) return true;
+  uint64_t t0;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  for (uint32_t i = 1;; ++i) {
+    if (bar_try(bar, parity)) return true;
+    if ((i & 63) == 0) {
+      uint64_t t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      if (t - t0 > limit_ns) return false;
+    }
+  }
+}
+
+// The tile ring of one CTA over its share of a tensor's tiles (tile i of the
+// CTA = sl.cta + i * sl.ncta): thread 0 keeps the next kTmaStages - 1 tiles
+// loading; fn(tile, smem of the tile) runs on every thread.  Returns false
+// after a wait ran out (error recorded, loads in flight drained).
+template <typename F>
+__device__ bool tma_tile_loop(const CUtensorMap* map, const QTensor& q, const Slice sl,
+                              uint8_t* smem, uint32_t* err, F&& fn) {
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTmaStages * kTmaTileBytes);
+  __shared__ int abort_flag;
+  const uint32_t ntc = (uint32_t)((q.cols + kTmaCols - 1) / kTmaCols);
+  const uint32_t ntiles = (uint32_t)((q.rows + kTmaRows - 1) / kTmaRows) * ntc;
+  const uint32_t mine = sl.cta < ntiles ? (ntiles - sl.cta + sl.ncta - 1) / sl.ncta : 0u;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kTmaStages; ++i)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&full[i])) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    abort_flag = 0;
+  }
+  __syncthreads();
+  auto issue = [&](uint32_t i) {  // thread 0: tile i of this CTA into slot i % kTmaStages
+    const uint32_t t = sl.cta + i * sl.ncta;
+    const uint32_t bar = smem_addr(&full[i % kTmaStages]);
+    const int32_t c0 = (int32_t)((t % ntc) * kTmaCols), r0 = (int32_t)((t / ntc) * kTmaRows);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+                 "r"(kTmaTileBytes)
+                 : "memory");
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(smem + (i % kTmaStages) * kTmaTileBytes)),
+        "l"((uint64_t)map), "r"(c0), "r"(r0), "r"(bar)
+        : "memory");
+  };
+  uint32_t issued = 0;
+  if (threadIdx.x == 0)
+    for (; issued < mine && issued < (uint32_t)kTmaStages - 1; ++issued) issue(issued);
+  bool ok = true;
+  for (uint32_t i = 0; i < mine; ++i) {
+    if (threadIdx.x == 0 && issued < mine) issue(issued++);  // the slot freed by tile i - 1
+    if (!bar_wait(smem_addr(&full[i % kTmaStages]), (i / kTmaStages) & 1u, kTmaWaitNs)) {
+      abort_flag = 1;
+    } else {
+      fn(sl.cta + i * sl.ncta, smem + (i % kTmaStages) * kTmaTileBytes);
+    }
+    __syncthreads();  // every thread is done with slot i before it is refilled
+    if (abort_flag) {
+      ok = false;
+      break;
+    }
+  }
+  if (!ok && threadIdx.x == 0) {
+    atomicOr(err, kDevErrTimeout);
+    // loads still in flight: the unconsumed tiles are among the last
+    // kTmaStages issued (tiles before those were waited for)
+    for (uint32_t j = issued > (uint32_t)kTmaStages ? issued - kTmaStages : 0u; j < issued; ++j)
+      bar_wait(smem_addr(&full[j % kTmaStages]), (j / kTmaStages) & 1u, kTmaDrainNs);
+  }
+  return ok;
+}
+
+// This thread's 16 words of a tile: rows 16 g .. 16 g + 15 of column pair cp
+// (word j = row j, both columns).  With the transform, the signs s_j are
+// applied here, to both columns of a row at once.
+template <bool RHT>
+__device__ __forceinline__ void tile_words(const uint8_t* tile, uint32_t mask, uint32_t w[16]) {
+  const uint32_t cp = threadIdx.x & 63, g = threadIdx.x >> 6;
+  const uint32_t* tw = reinterpret_cast<const uint32_t*>(tile) + (16 * g) * (kTmaCols / 2) + cp;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    w[j] = tw[j * (kTmaCols / 2)];
+    if (RHT) w[j] ^= ((mask >> j) & 1u) * 0x80008000u;
+  }
+}
+// The column block h (0: even column, 1: odd column) of those words, widened,
+// with the butterflies of the transform along rows when RHT.
+template <bool RHT>
+__device__ __forceinline__ void column_block(const uint32_t w[16], int h, float v[16]) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(h ? (w[j] & 0xFFFF0000u) : (w[j] << 16));
+  if (RHT) rht16_butterflies(v);
+}
+
+template <bool RHT>
+__global__ void __launch_bounds__(kThreads, 3)
+    amax_cols_tma_kernel(const __grid_constant__ QBatch p, const __grid_constant__ ColsMaps maps) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int t = blockIdx.y;
+  const QTensor& q = p.t[t];
+  const Slice sl{blockIdx.x, gridDim.x};
+  float m = 0.0f;
+  tma_tile_loop(&maps.m[t], q, sl, smem, p.err, [&](uint32_t, const uint8_t* tile) {
+    uint32_t w[16];
+    tile_words<RHT>(tile, p.mask, w);  // zero past the tensor's edges: no effect on the max
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float v[16];
+      column_block<RHT>(w, h, v);
+      m = fmaxf(m, absmax16(v));
+    }
+  });
+  m = block_reduce_max(m);
+  if (threadIdx.x == 0) p.partials[t * kMaxAmaxCtas + sl.cta] = m;
+  pdl_trigger();
+}
+
+template <bool RHT>
+__global__ void __launch_bounds__(kThreads, 2)
+    encode_cols_tma_kernel(const __grid_constant__ QBatch p, const __grid_constant__ ColsMaps maps,
+                           int ga) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int t = blockIdx.y;
+  const QTensor& q = p.t[t];
+  const Slice sl{blockIdx.x, gridDim.x};
+  float alpha;
+  if (p.gs_in) {
+    alpha = *p.gs_in;
+  } else {
+    pdl_wait();
+    alpha = alpha_from_amax(reduce_partials(p.partials + t * kMaxAmaxCtas, ga));
+  }
+  if (sl.cta == 0 && threadIdx.x == 0 && q.gs_out) *q.gs_out = alpha;
+  // per-warp queue of handed-back blocks; each entry carries the block's 16
+  // input values (bf16, element j in half j % 2 of word j / 2), so the redo
+  // reads shared memory, not the tile's rows in global memory again
+  __shared__ uint2 queue[kThreads / 32][kQueueCap];
+  __shared__ uint4 qdata[kThreads / 32][kQueueCap][2];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t qn = 0;  // same value on every lane
+  const uint32_t kb_total = (uint32_t)(q.rows >> 4);
+  const int64_t out_row_bytes = q.rows >> 1;
+  const FastDiv div_out = make_fastdiv(kb_total);
+  const bool fos = p.four_over_six != 0;
+  const ScaleCtx ctx = make_scale_ctx(alpha);
+  const uint32_t ntc = (uint32_t)((q.cols + kTmaCols - 1) / kTmaCols);
+  // queued entries hold the output block index c * kb_total + kb
+  auto drain = [&]() {
+    __syncwarp();
+    for (uint32_t i = lane; i < qn; i += 32) {
+      const uint2 it = queue[warp][i];
+      const uint4 d0 = qdata[warp][i][0], d1 = qdata[warp][i][1];
+      const uint32_t dw[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+      float v[16];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        v[2 * k] = __uint_as_float(dw[k] << 16);
+        v[2 * k + 1] = __uint_as_float(dw[k] & 0xFFFF0000u);
+      }
+      if (RHT) rht16_butterflies(v);  // signs already applied to the queued words
+      const uint32_t c = fastdiv(it.x, div_out), kb = it.x - c * kb_total;
+      redo_block(v, it.y, ctx, fos, q.codes + (int64_t)c * out_row_bytes + (int64_t)kb * 8,
+                 q.scales + sf_offset(c, kb, kb_total, p.sf_layout));
+    }
+    __syncwarp();
+    qn = 0;
+  };
+  tma_tile_loop(&maps.m[t], q, sl, smem, p.err, [&](uint32_t tile_id, const uint8_t* tile) {
+    uint32_t w[16];
+    tile_words<RHT>(tile, p.mask, w);
+    const uint32_t kb = (tile_id / ntc) * (kTmaRows / 16) + (threadIdx.x >> 6);
+    const int64_t c0 = (int64_t)(tile_id % ntc) * kTmaCols + 2 * (threadIdx.x & 63);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t c = c0 + h;
+      const bool valid = kb < kb_total && c < q.cols;
+      uint32_t st = kBlockDone, sc = 0u;
+      if (valid) {
+        float v[16];
+        column_block<RHT>(w, h, v);
+        uint64_t yy[8];
+        pairs_of(v, yy);
+        uint32_t lo, hi;
+        st = quantize_block16_pairs(yy, absmax16(v), ctx, fos, lo, hi, sc);
+        if (st == kBlockDone) store_codes(q.codes + c * out_row_bytes + (int64_t)kb * 8, lo, hi);
+        if (st != kBlockExact) q.scales[sf_offset(c, kb, kb_total, p.sf_layout)] = (uint8_t)sc;
+      }
+      const bool need = st != kBlockDone;
+      const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
+      if (need) {
+        const uint32_t slot = qn + __popc(m & ((1u << lane) - 1u));
+        queue[warp][slot] = make_uint2((uint32_t)c * kb_total + kb,
+                                       st == kBlockExact ? kRedoAll : sc);
+        uint32_t dw[8];  // column h's 16 values, two rows per word
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          dw[k] = h ? ((w[2 * k] >> 16) | (w[2 * k + 1] & 0xFFFF0000u))
+                    : ((w[2 * k] & 0xFFFFu) | (w[2 * k + 1] << 16));
+        qdata[warp][slot][0] = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+        qdata[warp][slot][1] = make_uint4(dw[4], dw[5], dw[6], dw[7]);
+      }
+      qn += __popc(m);
+    }
+    if (qn > kQueueCap - 64) drain();
+  });
+  drain();
+  if (p.sf_layout == 1) zero_sf_padding(q.scales, q.cols, kb_total, sl);
+}
+
 // Encode pass, 16x16 tiles.  A warp holds two adjacent tiles of one 16-row
 // band: lane l owns row (l & 15) of tile (l >> 4).  Tile max and tile error
 // reduce across the 16 lanes of a half-warp with xor shuffles 8, 4, 2, 1 --
@@ -453,7 +752,7 @@ __device__ void encode_2d(const QTensor& q, float alpha, const QBatch& p, uint2*
   const ScaleCtx ctx = make_scale_ctx(alpha);
   const FastDiv div = make_fastdiv(npair), div_blk = make_fastdiv(kbpr);
   // queued entries hold the block index r * kbpr + kb and the tile's scale
-  auto redo = [&](uint2 it) {
+  auto redo = [&](uint2 it, const uint4*) {
     const uint32_t r = fastdiv(it.x, div_blk), kb = it.x - r * kbpr;
     float v[16];
     load16(x + (int64_t)r * q.ld + (int64_t)kb * 16, v);
@@ -466,7 +765,7 @@ __device__ void encode_2d(const QTensor& q, float alpha, const QBatch& p, uint2*
     kb = tp * 2 + (lane >> 4);
     return kb < kbpr;
   };
-  WarpQueue wq{qbuf, 0u};
+  WarpQueue wq{qbuf, 0u, nullptr};
   const uint32_t ustride = sl.ncta * warps;
   uint32_t u = sl.cta * warps + (threadIdx.x >> 5);
   // the next unit's block is loaded before the current one is encoded
@@ -594,11 +893,22 @@ __global__ void __launch_bounds__(kThreads) finalize_kernel(const __grid_constan
 // the global scale is given).
 // Resident CTAs per SM the encode kernels are compiled for: the row-axis mode
 // holds two 16-element columns per thread and needs the larger register file.
-template <int MODE>
-constexpr int encode_min_blocks() { return MODE == kModeCols ? 2 : 3; }
+#ifndef NVFP4_ROWS_PACKED
+#define NVFP4_ROWS_PACKED 1
+#endif
+#ifndef NVFP4_ROWS_MIN_BLOCKS
+#define NVFP4_ROWS_MIN_BLOCKS 3
+#endif
+template <typename T, int MODE>
+constexpr int encode_min_blocks() {
+  return MODE == kModeCols ? 2
+         : (MODE == kModeRows && std::is_same<T, float>::value) ? 2
+         : (MODE == kModeRows || MODE == kModeMixed) ? NVFP4_ROWS_MIN_BLOCKS
+                                                     : 3;
+}
 
 template <typename T, int MODE, bool RHT>
-__global__ void __launch_bounds__(kThreads, encode_min_blocks<MODE>()) encode_kernel(const __grid_constant__ QBatch p, int ga) {
+__global__ void __launch_bounds__(kThreads, encode_min_blocks<T, MODE>()) encode_kernel(const __grid_constant__ QBatch p, int ga) {
   Slice sl{blockIdx.x, gridDim.x};
   int t = blockIdx.y;
   if constexpr (MODE == kModeMixed) {
@@ -614,16 +924,18 @@ __global__ void __launch_bounds__(kThreads, encode_min_blocks<MODE>()) encode_ke
   }
   if (sl.cta == 0 && threadIdx.x == 0 && p.t[t].gs_out) *p.t[t].gs_out = alpha;
   __shared__ uint2 queue[kThreads / 32][kQueueCap];
+  __shared__ uint4 qraw[kThreads / 32][2 * kQueueCap];
   uint2* qbuf = queue[threadIdx.x >> 5];
+  uint4* qdata = qraw[threadIdx.x >> 5];
   if constexpr (MODE == kModeRows) {
-    encode_rows<T, RHT>(p.t[t], alpha, p, qbuf, sl);
+    encode_rows<T, RHT>(p.t[t], alpha, p, qbuf, qdata, sl);
   } else if constexpr (MODE == kModeCols) {
     encode_cols<T, RHT>(p.t[t], alpha, p, qbuf, sl);
   } else if constexpr (MODE == kMode2D) {
     encode_2d<T>(p.t[t], alpha, p, qbuf, sl);
   } else {
     if (p.two_d_of[t]) encode_2d<T>(p.t[t], alpha, p, qbuf, sl);
-    else encode_rows<T, false>(p.t[t], alpha, p, qbuf, sl);
+    else encode_rows<T, false>(p.t[t], alpha, p, qbuf, qdata, sl);
   }
 }
 
@@ -871,7 +1183,7 @@ cudaError_t launch_mode(const QBatch& b, cudaStream_t s) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, encode_kernel<T, MODE, RHT>, kThreads,
                                                       0) != cudaSuccess ||
         o < 1)
-      o = encode_min_blocks<MODE>();
+      o = encode_min_blocks<T, MODE>();
     return o;
   }();
   uint64_t cap = (uint64_t)num_sms() * (uint64_t)occ / (uint64_t)b.n;
@@ -881,11 +1193,96 @@ cudaError_t launch_mode(const QBatch& b, cudaStream_t s) {
   return launch_ex(encode_kernel<T, MODE, RHT>, dim3(gx, b.n), s, !b.gs_in, b, ga);
 }
 
+typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                      const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                      const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                      CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// One 64 x 128 tile map per bf16 tensor of the batch (zero fill past the
+// edges); false if the driver refuses one.
+bool make_cols_maps(const QBatch& b, ColsMaps& maps) {
+  TensorMapEncodeFn fn = (TensorMapEncodeFn)tensor_map_encoder();
+  if (!fn) return false;
+  for (int i = 0; i < b.n; ++i) {
+    const QTensor& q = b.t[i];
+    if (q.rows == 0 || q.cols == 0) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)q.cols, (cuuint64_t)q.rows};
+    cuuint64_t strides[1] = {(cuuint64_t)q.ld * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kTmaCols, (cuuint32_t)kTmaRows};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&maps.m[i], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(q.x), dims, strides,
+           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+  }
+  return true;
+}
+
+template <typename K>
+cudaError_t launch_maps(K kern, dim3 grid, cudaStream_t s, bool pdl, const QBatch& b,
+                        const ColsMaps& maps, int ga, bool with_ga) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kTmaSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (with_ga) return cudaLaunchKernelEx(&cfg, (void (*)(QBatch, ColsMaps, int))kern, b, maps, ga);
+  return cudaLaunchKernelEx(&cfg, (void (*)(QBatch, ColsMaps))kern, b, maps);
+}
+
+// Row-axis quantization of bf16 tensors through the TMA-staged kernels;
+// returns cudaErrorNotSupported (nothing launched) when a map cannot be made.
+template <bool RHT>
+cudaError_t launch_cols_tma(const QBatch& b, cudaStream_t s) {
+  ColsMaps maps;  // copied into the launch parameters
+  if (!make_cols_maps(b, maps)) return cudaErrorNotSupported;
+  static const bool attrs_ok = [] {
+    return cudaFuncSetAttribute(amax_cols_tma_kernel<RHT>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kTmaSmemBytes) == cudaSuccess &&
+           cudaFuncSetAttribute(encode_cols_tma_kernel<RHT>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kTmaSmemBytes) == cudaSuccess;
+  }();
+  if (!attrs_ok) return cudaErrorNotSupported;
+  uint64_t tiles = 0;
+  for (int i = 0; i < b.n; ++i) {
+    const QTensor& q = b.t[i];
+    const uint64_t t = (uint64_t)((q.rows + kTmaRows - 1) / kTmaRows) *
+                       (uint64_t)((q.cols + kTmaCols - 1) / kTmaCols);
+    tiles = t > tiles ? t : tiles;
+  }
+  int ga = 0;
+  if (!b.gs_in) {
+    uint64_t cap = (uint64_t)num_sms() * 3 / (uint64_t)b.n;
+    if (cap > (uint64_t)kMaxAmaxCtas) cap = kMaxAmaxCtas;
+    if (cap < 1) cap = 1;
+    ga = (int)(tiles < cap ? (tiles < 1 ? 1 : tiles) : cap);
+    cudaError_t e = launch_maps(amax_cols_tma_kernel<RHT>, dim3(ga, b.n), s, false, b, maps, 0, false);
+    if (e != cudaSuccess) return e;
+    if (b.amax_only) return launch_ex(finalize_kernel, dim3(b.n), s, true, b, ga);
+  }
+  uint64_t cap = (uint64_t)num_sms() * 2 / (uint64_t)b.n;
+  if (cap < 1) cap = 1;
+  const unsigned gx = (unsigned)(tiles < cap ? (tiles < 1 ? 1 : tiles) : cap);
+  return launch_maps(encode_cols_tma_kernel<RHT>, dim3(gx, b.n), s, !b.gs_in, b, maps, ga, true);
+}
+
 template <typename T>
 cudaError_t launch_typed(const QBatch& b, cudaStream_t s) {
   if (b.two_d) return launch_mode<T, kMode2D, false>(b, s);
-  if (b.block_axis == 1)
+  if (b.block_axis == 1) {
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+      const cudaError_t e = b.rht ? launch_cols_tma<true>(b, s) : launch_cols_tma<false>(b, s);
+      if (e != cudaErrorNotSupported) return e;
+    }
     return b.rht ? launch_mode<T, kModeCols, true>(b, s) : launch_mode<T, kModeCols, false>(b, s);
+  }
   return b.rht ? launch_mode<T, kModeRows, true>(b, s) : launch_mode<T, kModeRows, false>(b, s);
 }
 
@@ -935,7 +1332,7 @@ cudaError_t launch_mixed_typed(QBatch& b, cudaStream_t s) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, encode_kernel<T, kModeMixed, false>,
                                                       kThreads, 0) != cudaSuccess ||
         o < 1)
-      o = encode_min_blocks<kModeMixed>();
+      o = encode_min_blocks<T, kModeMixed>();
     return o;
   }();
   const int32_t ga = split_ctas(wa, ca, b.n, (uint64_t)num_sms() * 3, b.amax_end);

@@ -238,6 +238,38 @@ def test_quantize_transposed(rht, layout):
         assert float(a.cpu()[0]) == np.float32(ref[2])
 
 
+def test_quantize_transposed_strided_batched_and_fp32():
+    """The row-axis path on a strided bf16 input (row stride 264 > 200
+    columns), two bf16 tensors of different shapes in one batched call, and
+    an fp32 input, each against the oracle."""
+    from nvfp4_block_scaled_20_b200 import capi
+    mask = synth.rht_sign_mask(0)
+    base = synth.activation(4, 3, 336, 264)
+    x = base[:, :200]
+    q = nv.quantize_1d(base.to(DEV)[:, :200], rht=True, mask=mask, block_axis=1)
+    assert_q_equal(q, oracle.quantize_1d(to_oracle(x), rht=True, mask=mask, block_axis=1,
+                                         sf_layout=1), "strided")
+    xs = [synth.activation(4, 5, 1040, 136).to(DEV), synth.activation(4, 6, 208, 384).to(DEV)]
+    outs = [nv.QTensor(*nv._alloc_q(t.shape[1], t.shape[0], 1, DEV), t.shape[1], t.shape[0], 1)
+            for t in xs]
+    ws = nv.workspace(2)
+    d = (capi.nvfp4_tensor_desc * 2)()
+    for i, (t, o) in enumerate(zip(xs, outs)):
+        d[i] = capi.nvfp4_tensor_desc(t.data_ptr(), None, o.codes.data_ptr(), o.scales.data_ptr(),
+                                      o.alpha.data_ptr(), t.shape[0], t.shape[1], t.stride(0))
+    qp = capi.nvfp4_qparams(1, 1, mask, 1, 1, 0, None)
+    st = capi.nvfp4_quantize_1d_batched(d, 2, capi.NVFP4_BF16, qp, ws.data_ptr(), ws.numel(),
+                                        torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    for t, o in zip(xs, outs):
+        assert_q_equal(o, oracle.quantize_1d(to_oracle(t), rht=True, mask=mask, block_axis=1,
+                                             sf_layout=1), "batched")
+    xf = synth.activation(4, 7, 272, 96, dtype=torch.float32)
+    q = nv.quantize_1d(xf.to(DEV), rht=True, mask=mask, block_axis=1)
+    assert_q_equal(q, oracle.quantize_1d(xf.numpy(), rht=True, mask=mask, block_axis=1,
+                                         sf_layout=1), "fp32")
+
+
 def test_quantize_rht_rows():
     mask = 0x1234
     x = synth.activation(7, 1, 144, 320)
