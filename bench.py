@@ -778,6 +778,29 @@ def measure_rows(nv, synth, torch, dev, stream, timed, pk, reps):
     out["steps"]["qkv"]["note"] = "mixed quantize of X and W, GEMM, bf16 Y"
     del xq, wq, qa, qb, yq
 
+    # ---------------- 4-bit Ulysses payload (one rank's side; the exchange itself
+    # needs several GPUs and is not timed here)
+    from nvfp4_block_scaled_20_b200 import ulysses
+    s_loc, heads, hd, world_sp = 8190, 24, 128, 4  # 32760 tokens over SP = 4
+    lay = ulysses.PayloadLayout(s_loc, heads, hd, world_sp)
+    qsh = synth.kv_tensor(5, 0, 0, heads=s_loc, tokens=heads, head_dim=hd, device=dev)
+    torch.cuda.synchronize(dev)
+    sbuf = torch.empty(lay.buffer_bytes, dtype=torch.uint8, device=dev)
+    uout = torch.empty((world_sp * s_loc * lay.heads_per_rank, hd), dtype=torch.bfloat16,
+                       device=dev)
+    ne_q = s_loc * heads * hd
+    out["next3_ulysses_payload"] = {
+        "pack_Q_8190x24x128": bw(lambda: ulysses.pack(qsh, lay, sbuf, stream=stream),
+                                 (4 + qout) * ne_q,
+                                 "quantize into the 4 destination segments (two passes)"),
+        "unpack_to_bf16": bw(lambda: ulysses.unpack(sbuf, lay, uout, stream=stream),
+                             (qout + 2) * ne_q, "dequantize the 4 received segments"),
+        "payload_bytes": lay.buffer_bytes, "bf16_bytes": 2 * ne_q,
+        "compression": round(2 * ne_q / lay.buffer_bytes, 3),
+        "note": "the NCCL all-to-all between the two is not measured: one GPU per run here",
+    }
+    del qsh, sbuf, uout
+
     # ---------------- context: the library's NVFP4 GEMM on the same shapes
     out["context_cublas_nvfp4_scaled_mm"] = library_ceiling(torch, dev, tc)
 

@@ -332,26 +332,20 @@ __host__ __device__ constexpr uint32_t instr_desc(int M, int N) {
   return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// GELU(tanh form) in fp32: 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))).
-// tanh from the identity tanh(u) = 1 - 2 / (exp(2u) + 1), with the exp and
-// the quotient from the __expf / __fdividef intrinsics: for |2u| < 18 their
-// relative errors (a few ulp, growing with |u|) move tanh by less than 2^-18
-// absolute, and beyond it exp(2u) is either so large that the quotient
-// vanishes under the fp32 rounding of 1 - q (tanh = 1) or so small that
-// 1 - 2/(e + 1) rounds to -1; overflow to +inf gives q = 0, tanh = 1.  So
-// |GELU_gpu(y) - GELU(y)| <= 0.5 |y| 2^-18 + a few fp32 roundings of y,
-// below 2^-17 |y| -- negligible against the GEMM's 1e-3 sum_k |a_k b_k|.
-__device__ __forceinline__ float tanh_via_exp(float u) {
-  const float e = __expf(2.0f * u);
-  return 1.0f - __fdividef(2.0f, e + 1.0f);
-}
-// sqrt(2/pi) (y + 0.044715 y^3) = y (k0 + k0 k1 y^2), and 0.5 y (1 + t) =
-// 0.5 y t + 0.5 y, with fused multiply-adds (fp32 rounding only).
+// GELU(tanh form) in fp32: 0.5 y (1 + tanh(u)), u = sqrt(2/pi) (y + 0.044715
+// y^3), evaluated as y * sigmoid(2u) = y / (1 + exp(-2u)) (the same function:
+// 1 + tanh(u) = 2 / (1 + exp(-2u))), with the __expf / __fdividef intrinsics.
+// For |2u| up to the point where the quotient saturates, their relative
+// errors (a few ulp of exp, growing with |2u|, and 2 ulp of the quotient) move
+// the result by less than 2^-18 |y|; exp(-2u) overflowing to +inf gives
+// -0 (GELU of a large negative y is below any fp32 of its magnitude's
+// scale), and __fdividef returning 0 for denominators above 2^126 does the
+// same.  So |GELU_gpu(y) - GELU(y)| < 2^-17 |y| -- negligible against the
+// GEMM's 1e-3 sum_k |a_k b_k|.
 __device__ __forceinline__ float gelu_tanh(float y) {
   const float k0 = 0.7978845608028654f, k01 = 0.7978845608028654f * 0.044715f;
   const float inner = y * fmaf(k01, y * y, k0);
-  const float hy = 0.5f * y;
-  return fmaf(hy, tanh_via_exp(inner), hy);
+  return __fdividef(y, 1.0f + __expf(-2.0f * inner));
 }
 
 struct Params {
