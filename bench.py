@@ -776,7 +776,18 @@ def measure_rows(nv, synth, torch, dev, stream, timed, pk, reps):
                                                               stream=stream), 2.0 * Mq * Nq * Kq)
     out["steps"]["qkv"] = tc(qkv_step, 2.0 * Mq * Nq * Kq)
     out["steps"]["qkv"]["note"] = "mixed quantize of X and W, GEMM, bf16 Y"
-    del xq, wq, qa, qb, yq
+    # the same projection with a rank-128, scale-1 adapter fused in (W4A4 + LoRA)
+    rl = 128
+    lu = synth.activation(22, 101, Mq, rl, n_out=0, std=0.5, device=dev)
+    lb = synth.weight(22, 102, Nq, rl, device=dev)
+    lscr = torch.empty(nv.capi.nvfp4_lora_scratch_bytes(Mq, rl), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize(dev)
+    lora = tc(lambda: nv.gemm_lora(qa, qb, lu, lb, 1.0, out=yq, ws=ws, scratch=lscr,
+                                   stream=stream), 2.0 * Mq * Nq * (Kq + rl))
+    lora["note"] = ("FP4 GEMM plus the rank-128 bf16 adapter product in the same launch "
+                    "(and the adapter input's scaling kernel); flops 2 M N (K + r)")
+    out["next4_gemm_lora"] = {"qkv_2640x9216x3072_rank128": lora}
+    del xq, wq, qa, qb, yq, lu, lb, lscr
 
     # ---------------- 4-bit Ulysses payload (one rank's side; the exchange itself
     # needs several GPUs and is not timed here)

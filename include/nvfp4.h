@@ -338,6 +338,41 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf,
                         int64_t ldo, int32_t epilogue, void* workspace,
                         size_t workspace_bytes, void* stream);
 
+/* Bytes of the scratch nvfp4_gemm_lora needs for an M-row activation and a
+ * rank-`rank` adapter (the scaled adapter input, bf16 [M, 2 rank]). */
+NVFP4_API size_t nvfp4_lora_scratch_bytes(int64_t M, int64_t rank);
+
+/* W4A4 linear layer with its low-rank adapter in one GEMM -- notes, section
+ * 3.4 "NVFP4 training and DMD LoRA" (the quantized LoRA linear: frozen NVFP4
+ * backbone, bf16 adapter, delta = (x A^T) B^T * scale, rank 128 and alpha 128
+ * in the released adapter) and explainer, section 3.4 (W ~ Dequant(Q(W0)) +
+ * (alpha/r) B A; the deployed layer keeps the branch separate):
+ *   out[m, n] = epi( a_alpha b_alpha sum_k a_mk sA b_nk sB
+ *                    + lora_scale * sum_j lora_u[m, j] lora_b[n, j] ).
+ * The adapter's product runs on the tensor cores in the same kernel, into the
+ * same fp32 accumulator as the FP4 product, after each tile's FP4 stages
+ * (tcgen05.mma kind::f16, bf16 x bf16): lora_u * lora_scale / (a_alpha
+ * b_alpha) is first written to scratch as the bf16 pair hi + lo (within 2^-17
+ * of the fp32 value), so one epilogue scaling by a_alpha b_alpha serves both
+ * terms.
+ *   FP4 operands, out, epilogue, workspace: as nvfp4_gemm.
+ *   lora_u   device bf16 [M, rank], row stride ldu: x A^T, the adapter's
+ *            first product (16-byte aligned, ldu * 2 a multiple of 16).
+ *   lora_b   device bf16 [N, rank], row stride ldl: B (same alignment).
+ *   rank     a multiple of 64, 64..1024; lora_scale finite (alpha / rank).
+ *   scratch  device, nvfp4_lora_scratch_bytes(M, rank) bytes, 16-byte
+ *            aligned; overwritten.
+ * lora_scale / (a_alpha b_alpha) must be finite. */
+NVFP4_API nvfp4_status nvfp4_gemm_lora(const uint8_t* a_codes, const uint8_t* a_sf,
+                                       const float* a_alpha, const uint8_t* b_codes,
+                                       const uint8_t* b_sf, const float* b_alpha, int64_t M,
+                                       int64_t N, int64_t K, const void* lora_u, int64_t ldu,
+                                       const void* lora_b, int64_t ldl, int64_t rank,
+                                       float lora_scale, void* scratch, size_t scratch_bytes,
+                                       void* out, int32_t out_dtype, int64_t ldo,
+                                       int32_t epilogue, void* workspace, size_t workspace_bytes,
+                                       void* stream);
+
 /* ------------------------------------------------------------ RHT ------- */
 
 /* Standalone 16-point RHT, y = 1/4 H16 diag(s) x on every 16-group along

@@ -16,7 +16,7 @@ from .capi import (NVFP4_BF16, NVFP4_EPI_AMAX, NVFP4_EPI_GELU_TANH, NVFP4_EPI_NO
                    NVFP4_SF_ROWMAJOR, NVFP4_SF_TCGEN05, NVFP4Error)
 
 __all__ = ["QTensor", "quantize_1d", "quantize_2d", "global_scale", "quantize_1d_batched",
-           "quantize_mixed",
+           "quantize_mixed", "gemm_lora",
            "dequantize", "dequantize_rows", "window_row_ranges", "transpose_2d", "gemm", "rht16", "workspace",
            "device_error", "capi"]
 
@@ -263,6 +263,33 @@ def gemm(a: QTensor, b: QTensor, out_dtype=None, epilogue=NVFP4_EPI_NONE, out=No
                          out.data_ptr(), code, out.stride(0), epilogue, ws.data_ptr(), ws.numel(),
                          _stream(stream))
     capi.check("nvfp4_gemm", st)
+    return out
+
+
+def gemm_lora(a: QTensor, b: QTensor, lora_u, lora_b, lora_scale, out_dtype=None,
+              epilogue=NVFP4_EPI_NONE, out=None, ws=None, scratch=None, stream=None):
+    """nvfp4_gemm_lora: out = a b^T (NVFP4) + lora_scale * lora_u lora_b^T, the
+    adapter branch (bf16 lora_u [M, r] = x A^T, lora_b [N, r]) fused into the
+    same GEMM."""
+    torch = _torch()
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    M, K = a.rows, a.cols
+    N = b.rows
+    rank = lora_u.shape[1]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=a.codes.device)
+    ws = workspace(0, a.codes.device) if ws is None else ws
+    if scratch is None:
+        scratch = torch.empty(capi.nvfp4_lora_scratch_bytes(M, rank), dtype=torch.uint8,
+                              device=a.codes.device)
+    code = NVFP4_BF16 if out.dtype == torch.bfloat16 else NVFP4_F32
+    st = capi.nvfp4_gemm_lora(a.codes.data_ptr(), a.scales.data_ptr(), a.alpha.data_ptr(),
+                              b.codes.data_ptr(), b.scales.data_ptr(), b.alpha.data_ptr(), M, N, K,
+                              lora_u.data_ptr(), lora_u.stride(0), lora_b.data_ptr(),
+                              lora_b.stride(0), rank, float(lora_scale), scratch.data_ptr(),
+                              scratch.numel(), out.data_ptr(), code, out.stride(0), epilogue,
+                              ws.data_ptr(), ws.numel(), _stream(stream))
+    capi.check("nvfp4_gemm_lora", st)
     return out
 
 

@@ -26,6 +26,7 @@ EXPORTED = [
     "nvfp4_transpose_2d",
     "nvfp4_gemm", "nvfp4_rht16", "nvfp4_get_device_error", "nvfp4_status_string",
     "nvfp4_convert_sweep", "nvfp4_set_wait_limit", "nvfp4_set_test_stall",
+    "nvfp4_lora_scratch_bytes", "nvfp4_gemm_lora",
 ]
 
 
@@ -77,6 +78,9 @@ _SIGS = {
     "nvfp4_convert_sweep": (_I32, [_I32, _U32, _I64, _V, _V]),
     "nvfp4_set_wait_limit": (_I32, [ctypes.c_uint64]),
     "nvfp4_set_test_stall": (_I32, [_I32]),
+    "nvfp4_lora_scratch_bytes": (_SZ, [_I64, _I64]),
+    "nvfp4_gemm_lora": (_I32, [_V, _V, _V, _V, _V, _V, _I64, _I64, _I64, _V, _I64, _V, _I64, _I64,
+                               ctypes.c_float, _V, _SZ, _V, _I32, _I64, _I32, _V, _SZ, _V]),
 }
 
 
@@ -165,6 +169,18 @@ def nvfp4_dequantize_rows(descs, n, row_ranges, n_ranges, out_dtype, sf_layout, 
 def nvfp4_gemm(a_codes, a_sf, a_alpha, b_codes, b_sf, b_alpha, M, N, K, out, out_dtype, ldo,
                epilogue, ws, ws_bytes, stream):
     return _call("nvfp4_gemm", a_codes, a_sf, a_alpha, b_codes, b_sf, b_alpha, M, N, K, out,
+                 out_dtype, ldo, epilogue, ws, ws_bytes, stream)
+
+
+def nvfp4_lora_scratch_bytes(M, rank):
+    return _call("nvfp4_lora_scratch_bytes", M, rank)
+
+
+def nvfp4_gemm_lora(a_codes, a_sf, a_alpha, b_codes, b_sf, b_alpha, M, N, K, lora_u, ldu, lora_b,
+                    ldl, rank, lora_scale, scratch, scratch_bytes, out, out_dtype, ldo, epilogue,
+                    ws, ws_bytes, stream):
+    return _call("nvfp4_gemm_lora", a_codes, a_sf, a_alpha, b_codes, b_sf, b_alpha, M, N, K,
+                 lora_u, ldu, lora_b, ldl, rank, lora_scale, scratch, scratch_bytes, out,
                  out_dtype, ldo, epilogue, ws, ws_bytes, stream)
 
 

@@ -328,10 +328,61 @@ nvfp4_status nvfp4_transpose_2d(const uint8_t* codes, const uint8_t* scales,
                                          out_scales, sf_layout_out, S(stream)));
 }
 
+namespace {
+nvfp4_status gemm_common(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_alpha,
+                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_alpha,
+                         int64_t M, int64_t N, int64_t K, void* out, int32_t out_dtype,
+                         int64_t ldo, int32_t epilogue, void* ws, size_t ws_bytes, void* stream,
+                         const GemmArgs* lora);
+}  // namespace
+
 nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_alpha,
                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_alpha,
                         int64_t M, int64_t N, int64_t K, void* out, int32_t out_dtype, int64_t ldo,
                         int32_t epilogue, void* ws, size_t ws_bytes, void* stream) {
+  return gemm_common(a_codes, a_sf, a_alpha, b_codes, b_sf, b_alpha, M, N, K, out, out_dtype, ldo,
+                     epilogue, ws, ws_bytes, stream, nullptr);
+}
+
+size_t nvfp4_lora_scratch_bytes(int64_t M, int64_t rank) {
+  return (M > 0 && rank > 0) ? (size_t)M * (size_t)rank * 4u : 0u;
+}
+
+nvfp4_status nvfp4_gemm_lora(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_alpha,
+                             const uint8_t* b_codes, const uint8_t* b_sf, const float* b_alpha,
+                             int64_t M, int64_t N, int64_t K, const void* lora_u, int64_t ldu,
+                             const void* lora_b, int64_t ldl, int64_t rank, float lora_scale,
+                             void* scratch, size_t scratch_bytes, void* out, int32_t out_dtype,
+                             int64_t ldo, int32_t epilogue, void* ws, size_t ws_bytes,
+                             void* stream) {
+  if (!lora_u || !lora_b || !scratch) return NVFP4_ERR_INVALID_ARG;
+  if (rank < 64 || rank > 1024 || rank % 64 || ldu < rank || ldl < rank) return NVFP4_ERR_SHAPE;
+  if (!(lora_scale == lora_scale) || lora_scale > 3.0e38f || lora_scale < -3.0e38f)
+    return NVFP4_ERR_INVALID_ARG;  // finite scale
+  if (!aligned(lora_u, 16) || !aligned(lora_b, 16) || !aligned(scratch, 16) || (ldu * 2) % 16 ||
+      (ldl * 2) % 16)
+    return NVFP4_ERR_ALIGN;
+  if (scratch_bytes < nvfp4_lora_scratch_bytes(M, rank)) return NVFP4_ERR_WORKSPACE;
+  GemmArgs l{};
+  l.lora_u = lora_u;
+  l.lora_b = lora_b;
+  l.ldu = ldu;
+  l.ldl = ldl;
+  l.rank = rank;
+  l.lora_scale = lora_scale;
+  l.u_scaled = scratch;
+  return gemm_common(a_codes, a_sf, a_alpha, b_codes, b_sf, b_alpha, M, N, K, out, out_dtype, ldo,
+                     epilogue, ws, ws_bytes, stream, &l);
+}
+
+}  // extern "C"
+
+namespace {
+nvfp4_status gemm_common(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_alpha,
+                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_alpha,
+                         int64_t M, int64_t N, int64_t K, void* out, int32_t out_dtype,
+                         int64_t ldo, int32_t epilogue, void* ws, size_t ws_bytes, void* stream,
+                         const GemmArgs* lora) {
   if (!a_codes || !a_sf || !a_alpha || !b_codes || !b_sf || !b_alpha || !out)
     return NVFP4_ERR_INVALID_ARG;
   if (!dtype_ok(out_dtype)) return NVFP4_ERR_INVALID_ARG;
@@ -362,11 +413,27 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
   g.amax_partials = want_amax ? partials(ws) : nullptr;
   g.wait_limit_ns = gemm_wait_limit_ns();
   g.stall = gemm_test_stall();
+  g.lora_u = nullptr;
+  g.lora_b = nullptr;
+  g.rank = 0;
+  g.u_scaled = nullptr;
+  if (lora) {
+    g.lora_u = lora->lora_u;
+    g.lora_b = lora->lora_b;
+    g.ldu = lora->ldu;
+    g.ldl = lora->ldl;
+    g.rank = lora->rank;
+    g.lora_scale = lora->lora_scale;
+    g.u_scaled = lora->u_scaled;
+  }
   bool unsupported = false;
   int e = launch_gemm(g, S(stream), &unsupported);
   if (unsupported) return NVFP4_ERR_UNSUPPORTED;
   return e == 0 ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
+}  // namespace
+
+extern "C" {
 
 nvfp4_status nvfp4_rht16(const void* x, int32_t dtype, int64_t rows, int64_t cols, int64_t ld,
                          int32_t block_axis, uint32_t sign_mask, float* out, void* stream) {

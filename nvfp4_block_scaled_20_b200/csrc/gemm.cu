@@ -261,6 +261,15 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uin
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
+// bf16 x bf16 -> fp32 MMA of a CTA pair (the LoRA branch), K = 16 per call.
+__device__ __forceinline__ void tc_mma_pair_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t r[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
@@ -331,6 +340,13 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t addr) {
 __host__ __device__ constexpr uint32_t instr_desc(int M, int N) {
   return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// Instruction descriptor, kind::f16 with bf16 A and B (format 1 in bits 7-9
+// and 10-12), fp32 accumulation (bits 4-5 = 1), K-major A and B, N >> 3 in
+// bits 17-22, M >> 4 in bits 24-28.
+__host__ __device__ constexpr uint32_t instr_desc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
 
 // GELU(tanh form) in fp32: 0.5 y (1 + tanh(u)), u = sqrt(2/pi) (y + 0.044715
 // y^3), evaluated as y * sigmoid(2u) = y / (1 + exp(-2u)) (the same function:
@@ -366,6 +382,10 @@ struct Params {
   float* amax_partials;
   uint64_t wait_limit_ns;  // bound of each pipeline wait
   int32_t stall;           // test hook: the MMA issuer first waits on a barrier nothing completes
+  // LoRA branch: lora_kt extra ring stages per tile after the FP4 stages,
+  // each a 128-byte column chunk (64 bf16) of the scaled adapter input U'
+  // [M, 2r] (hi and lo halves) and of B_lora [N, r] (chunk c mod lora_kt / 2)
+  int32_t lora_kt;
 };
 
 // Tile t of the grouped raster -> (tile row, tile column).
@@ -428,7 +448,8 @@ __device__ __forceinline__ void stage16(const Params& p, uint8_t* chunk, int lan
 
 __global__ void __launch_bounds__(kNumThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ Params p) {
+                const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmU,
+                const __grid_constant__ CUtensorMap tmL, const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = smem;
@@ -460,6 +481,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   const int num_m = (p.M + 2 * BM - 1) / (2 * BM), num_n = (p.N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
   const int num_kt = (p.K + BK - 1) / BK;
+  const int total_kt = num_kt + p.lora_kt;  // FP4 stages, then the LoRA stages of a tile
   const int kgroups = p.K / 64;  // 4-block scale groups per 128-row band
   const int mbands_total = (p.M + 127) / 128, nbands_total = (p.N + 127) / 128;
 
@@ -512,7 +534,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         tile_coords(t, num_m, num_n, mt, nt);
         const int m0 = mt * 2 * BM + (int)rank * BM, nb0 = nt * BN + (int)rank * (BN / 2);
         const int mband = mt * 2 + (int)rank;
-        for (int kt = 0; kt < num_kt; ++kt, ++it) {
+        for (int kt = 0; kt < total_kt; ++kt, ++it) {
           const int s = it % kStages;
           const uint32_t round = it / kStages;
           if (!mbar_wait(smem_u32(&empty[s]), (round & 1u) ^ 1u, abort_flag, p.wait_limit_ns)) {
@@ -521,6 +543,15 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           }
           const uint32_t fb = map_to_rank(smem_u32(&full[s]), 0);
           if (leader) mbar_expect_tx(smem_u32(&full[s]), 2 * (kABytes + kBBytes));
+          if (kt >= num_kt) {
+            // LoRA stage: 128-byte chunks of U' and B_lora, no scale atoms
+            const int c = kt - num_kt;
+            tma_load_2d_pair(smem_u32(sA + s * kABytes), &tmU, c * BK_BYTES, m0, fb);
+            tma_load_2d_pair(smem_u32(sB + s * kBBytes), &tmL, (c % (p.lora_kt / 2)) * BK_BYTES,
+                             nb0, fb);
+            mbar_expect_tx(smem_u32(&sf_in[s]), 0u);
+            continue;
+          }
           tma_load_2d_pair(smem_u32(sA + s * kABytes), &tmA, kt * BK_BYTES, m0, fb);
           tma_load_2d_pair(smem_u32(sB + s * kBBytes), &tmB, kt * BK_BYTES, nb0, fb);
           const int atoms = min(4, kgroups - kt * 4);
@@ -593,7 +624,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         }
         tc_fence_after();
         const uint32_t t_acc = tmem + (b ? kAcc1Col : 0u);
-        for (int kt = 0; kt < num_kt; ++kt, ++it) {
+        for (int kt = 0; kt < total_kt; ++kt, ++it) {
           const int s = it % kStages;
           const uint32_t slot = it % kSfSlots;
           if (!mbar_wait(smem_u32(&full[s]), (it / kStages) & 1u, abort_flag, p.wait_limit_ns) ||
@@ -602,13 +633,22 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             break;
           }
           tc_fence_after();
-          const int nmma = min(4, (p.K - kt * BK) / MMA_K);
           const uint32_t a_base = smem_u32(sA + s * kABytes);
           const uint32_t b_base = smem_u32(sB + s * kBBytes);
-          const uint32_t t_sf = tmem + kSfSlotCol + slot * kSfSlotCols;
-          for (int k = 0; k < nmma; ++k)
-            tc_mma_pair(t_acc, operand_desc(a_base + 32 * k), operand_desc(b_base + 32 * k), idesc,
-                        t_sf + 4 * k, t_sf + 16 + 8 * k, (kt > 0 || k > 0) ? 1u : 0u);
+          if (kt >= num_kt) {
+            // LoRA stage: four bf16 MMAs (K = 16, 32 bytes of each row) into the
+            // same accumulator, which the FP4 stages have initialised
+            constexpr uint32_t idesc16 = instr_desc_bf16(2 * BM, BN);
+            for (int k = 0; k < 4; ++k)
+              tc_mma_pair_bf16(t_acc, operand_desc(a_base + 32 * k), operand_desc(b_base + 32 * k),
+                               idesc16, 1u);
+          } else {
+            const int nmma = min(4, (p.K - kt * BK) / MMA_K);
+            const uint32_t t_sf = tmem + kSfSlotCol + slot * kSfSlotCols;
+            for (int k = 0; k < nmma; ++k)
+              tc_mma_pair(t_acc, operand_desc(a_base + 32 * k), operand_desc(b_base + 32 * k),
+                          idesc, t_sf + 4 * k, t_sf + 16 + 8 * k, (kt > 0 || k > 0) ? 1u : 0u);
+          }
           tc_commit_pair(smem_u32(&empty[s]));
           tc_commit_pair(smem_u32(&sf_empty[slot]));
         }
@@ -730,7 +770,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     uint32_t it = 0;
     bool ok = true;
     for (int t = pair; t < num_tiles && ok; t += num_pairs) {
-      for (int kt = 0; kt < num_kt; ++kt, ++it) {
+      for (int kt = 0; kt < total_kt; ++kt, ++it) {
         const int s = it % kStages;
         const uint32_t slot = it % kSfSlots;
         if (!mbar_wait(smem_u32(&sf_in[s]), (it / kStages) & 1u, abort_flag, p.wait_limit_ns) ||
@@ -738,6 +778,15 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                        p.wait_limit_ns)) {
           ok = false;
           break;
+        }
+        if (kt >= num_kt) {
+          // LoRA stage: no scales; hand the stage and the slot on unchanged
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(smem_u32(&empty[s]));
+            mbar_arrive_leader(smem_u32(&sf_full[slot]), leader);
+          }
+          continue;
         }
         tc_fence_after();
         uint32_t ra[16], rb[32];
@@ -784,6 +833,41 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   }
 }
 
+// The LoRA branch's adapter input, scaled into the accumulator's units: the
+// epilogue multiplies the whole accumulator by a_alpha * b_alpha, so the
+// bf16 MMAs must add u * c with c = scale / (a_alpha * b_alpha).  u * c (fp32)
+// is split into hi = bf16(u c) and lo = bf16(u c - hi), written side by side
+// as one [M, 2 rank] bf16 row each; hi + lo is within 2^-17 of u c, and the
+// MMAs' products of bf16 values are exact in fp32.  One thread per 8
+// consecutive elements of a row.
+__global__ void __launch_bounds__(256)
+    lora_prescale_kernel(const __nv_bfloat16* u, int64_t ldu, int64_t M, int64_t rank,
+                         const float* a_alpha, const float* b_alpha, float scale,
+                         __nv_bfloat16* out) {
+  const float c = __fdiv_rn(scale, __fmul_rn(*a_alpha, *b_alpha));
+  const int64_t groups = rank / 8, n = M * groups;
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t m = g / groups, j = (g - m * groups) * 8;
+    const uint4 raw = *reinterpret_cast<const uint4*>(u + m * ldu + j);
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float a = __fmul_rn(__uint_as_float(w[k] << 16), c);
+      const float b = __fmul_rn(__uint_as_float(w[k] & 0xFFFF0000u), c);
+      const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+      const float ha = __bfloat162float(h.x), hb = __bfloat162float(h.y);
+      const __nv_bfloat162 l = __floats2bfloat162_rn(__fsub_rn(a, ha), __fsub_rn(b, hb));
+      hi[k] = *reinterpret_cast<const uint32_t*>(&h);
+      lo[k] = *reinterpret_cast<const uint32_t*>(&l);
+    }
+    __nv_bfloat16* row = out + m * 2 * rank;
+    *reinterpret_cast<uint4*>(row + j) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(row + rank + j) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+}
+
 // --------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -791,6 +875,22 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() { return (EncodeTiledFn)tensor_map_encoder(); }
+
+// A matrix of `rows` rows of `row_bytes` bytes (row stride stride_bytes) as
+// 128-byte x box_rows tiles, 128-byte swizzle, zero fill past the edges.
+bool make_rows_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes,
+                   int64_t stride_bytes, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)stride_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)BK_BYTES, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 // Codes [rows, K/2] bytes, box = 128 bytes x box_rows rows, 128-byte swizzle,
 // out-of-bounds rows / columns read as zero.
@@ -842,11 +942,30 @@ bool make_out_map(CUtensorMap* map, void* out, int64_t M, int64_t N, int64_t ldo
 }
 
 int launch_persistent(const GemmArgs& a, cudaStream_t s) {
-  CUtensorMap tmA, tmB, tmOut;
+  CUtensorMap tmA, tmB, tmOut, tmU, tmL;
   if (!make_out_map(&tmOut, a.out, a.M, a.N, a.ldo, a.out_bf16 != 0))
     return (int)cudaErrorInvalidValue;
   if (!make_codes_map(&tmA, a.a_codes, a.M, a.K, BM)) return (int)cudaErrorInvalidValue;
   if (!make_codes_map(&tmB, a.b_codes, a.N, a.K, BN / 2)) return (int)cudaErrorInvalidValue;
+  int32_t lora_kt = 0;
+  if (a.rank > 0) {
+    // the scaled adapter input first (the GEMM waits for it: programmatic launch)
+    const int64_t groups = a.M * (a.rank / 8);
+    int64_t grid = (groups + 255) / 256;
+    if (grid > (int64_t)num_sms() * 8) grid = (int64_t)num_sms() * 8;
+    lora_prescale_kernel<<<(unsigned)(grid < 1 ? 1 : grid), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(a.lora_u), a.ldu, a.M, a.rank, a.a_alpha, a.b_alpha,
+        a.lora_scale, static_cast<__nv_bfloat16*>(a.u_scaled));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return (int)e;
+    if (!make_rows_map(&tmU, a.u_scaled, a.M, 4 * a.rank, 4 * a.rank, BM) ||
+        !make_rows_map(&tmL, a.lora_b, a.N, 2 * a.rank, 2 * a.ldl, BN / 2))
+      return (int)cudaErrorInvalidValue;
+    lora_kt = (int32_t)(a.rank / 32);  // 2 rank bf16 of U' per row = rank / 32 chunks of 128 B
+  } else {
+    tmU = tmA;  // unused
+    tmL = tmB;
+  }
   Params p;
   p.a_sf = a.a_sf;
   p.b_sf = a.b_sf;
@@ -863,6 +982,7 @@ int launch_persistent(const GemmArgs& a, cudaStream_t s) {
   p.err = a.err;
   p.wait_limit_ns = a.wait_limit_ns;
   p.stall = a.stall;
+  p.lora_kt = lora_kt;
   // resident pairs: one pair per two SMs where the GPU's layout allows
   static const int max_pairs = [] {
     if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -880,7 +1000,7 @@ int launch_persistent(const GemmArgs& a, cudaStream_t s) {
   const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
   cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = pair_config(dim3(2 * pairs), s, attr);
-  return (int)cudaLaunchKernelEx(&cfg, gemm_kernel, tmA, tmB, tmOut, p);
+  return (int)cudaLaunchKernelEx(&cfg, gemm_kernel, tmA, tmB, tmOut, tmU, tmL, p);
 }
 
 }  // namespace

@@ -86,6 +86,14 @@ struct GemmArgs {
   float* amax_partials;  // non-null: per-CTA output amax (kMaxAmaxCtas slots)
   uint64_t wait_limit_ns;  // bound of each pipeline wait before the kernel gives up
   int32_t stall;           // test hook (nvfp4_set_test_stall)
+  // LoRA branch (rank 0: none): u [M, rank] bf16 (row stride ldu), bl [N, rank]
+  // bf16 (row stride ldl), out += scale * u bl^T; u_scaled: bf16 [M, 2 rank]
+  // scratch for the scaled adapter input
+  const void* lora_u;
+  const void* lora_b;
+  int64_t ldu, ldl, rank;
+  float lora_scale;
+  void* u_scaled;
 };
 
 // Default bound of a GEMM pipeline wait, and the process-wide settings

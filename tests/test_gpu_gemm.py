@@ -198,3 +198,89 @@ def test_gelu_epilogue_on_exact_products():
     bad = np.argwhere(np.abs(got - want) > tol)
     assert bad.size == 0, "%d outputs, first y=%r gpu=%r ref=%r" % (
         len(bad), y[tuple(bad[0])], got[tuple(bad[0])], want[tuple(bad[0])])
+
+
+# ------------------------------------------------------------ W4A4 + LoRA
+def _lora_inputs(seed, M, N, r):
+    u = synth.activation(seed, 101, M, r, n_out=0, std=0.5)     # x A^T, bf16 [M, r]
+    bl = synth.weight(seed, 102, N, r)                           # B, bf16 [N, r]
+    return u, bl
+
+
+@pytest.mark.parametrize("M,N,K,r,scale,out_dtype,epi", [
+    (64, 128, 256, 128, 1.0, torch.float32, nv.NVFP4_EPI_NONE),      # the tiny linear's shape
+    (200, 272, 320, 64, 0.5, torch.bfloat16, nv.NVFP4_EPI_NONE),     # ragged M, N; partial K
+    (300, 384, 512, 128, 2.0, torch.bfloat16, nv.NVFP4_EPI_GELU_TANH),
+    (257, 512, 3072, 192, -0.75, torch.float32, nv.NVFP4_EPI_NONE),
+])
+def test_gemm_with_fused_lora_branch(M, N, K, r, scale, out_dtype, epi):
+    """out = a b^T (NVFP4) + scale * u bl^T in one GEMM launch against the
+    oracle's fp64 GEMM plus its LoRA branch (notes, section 3.4: the quantized
+    LoRA linear), |gpu - oracle| <= 1e-3 * (sum |a b| + |scale| sum |u bl|)."""
+    x = synth.activation(20, M, M, K)
+    w = synth.weight(20, N, N, K)
+    aref = oracle.quantize_1d(to_oracle(x), sf_layout=oracle.SF_TCGEN05)
+    bref = oracle.quantize_2d(to_oracle(w), sf_layout=oracle.SF_TCGEN05)
+    u, bl = _lora_inputs(21, M, N, r)
+    ws = nv.workspace(0)
+    out = nv.gemm_lora(upload(aref, M, K), upload(bref, N, K), u.to(DEV), bl.to(DEV), scale,
+                       out_dtype=out_dtype, epilogue=epi, ws=ws)
+    torch.cuda.synchronize()
+    assert nv.device_error(ws) == 0
+    y, s = oracle_gemm_ref(aref, bref, M, N, K)
+    y, s = oracle.lora_add(y, s, to_oracle(u), to_oracle(bl), scale)
+    gelu = epi == nv.NVFP4_EPI_GELU_TANH
+    if gelu:
+        y = np.vectorize(oracle.gelu_tanh)(y)
+    got = out.float().cpu().numpy().astype(np.float64)
+    tol = gemm_tolerance(y, s, out_dtype == torch.bfloat16, gelu)
+    bad = np.argwhere(np.abs(got - y) > tol)
+    assert bad.size == 0, "%d outputs out of tolerance, first %s: gpu=%r ref=%r tol=%r" % (
+        len(bad), bad[0], got[tuple(bad[0])], y[tuple(bad[0])], tol[tuple(bad[0])])
+    # the branch is really there: without it the result is far outside tolerance
+    y0, s0 = oracle_gemm_ref(aref, bref, M, N, K)
+    if gelu:
+        y0 = np.vectorize(oracle.gelu_tanh)(y0)
+    assert (np.abs(got - y0) > tol).mean() > 0.5
+
+
+def test_gemm_lora_qkv_shape_sampled():
+    """The DiT QKV projection with a rank-128, scale-1 adapter (the released
+    adapter's rank and alpha): the fused GEMM on a sampled grid of outputs."""
+    x, w = synth.qkv_linear(DEV)
+    M, K = x.shape
+    N = w.shape[0]
+    ws = nv.workspace(2)
+    qa, qb = nv.quantize_mixed([x, w], [False, True], ws=ws)
+    u, bl = _lora_inputs(22, M, N, 128)
+    out = nv.gemm_lora(qa, qb, u.to(DEV), bl.to(DEV), 1.0, out_dtype=torch.bfloat16, ws=ws)
+    torch.cuda.synchronize()
+    assert nv.device_error(ws) == 0
+    rng = np.random.default_rng(23)
+    mi = np.unique(np.concatenate([rng.choice(M, 40, replace=False), [0, M - 1]]))
+    ni = np.unique(np.concatenate([rng.choice(N // 16, 3, replace=False) * 16, [0]]))
+    ni = (ni[:, None] + np.arange(16)[None, :]).reshape(-1)
+    ax, aw = float(qa.alpha.cpu()[0]), float(qb.alpha.cpu()[0])
+    xr = oracle.quantize_1d(to_oracle(x.cpu()[torch.from_numpy(mi)]), alpha_in=ax)
+    wr = oracle.quantize_2d(to_oracle(w.cpu()[torch.from_numpy(ni)]), alpha_in=aw)
+    y, s = oracle.gemm((xr[0], xr[1], ax, oracle.SF_ROWMAJOR), (wr[0], wr[1], aw, oracle.SF_ROWMAJOR),
+                       len(mi), len(ni), K)
+    y, s = oracle.lora_add(y, s, to_oracle(u)[mi], to_oracle(bl)[ni], 1.0)
+    got = out.index_select(0, torch.from_numpy(mi).to(DEV)).index_select(
+        1, torch.from_numpy(ni).to(DEV)).float().cpu().numpy().astype(np.float64)
+    tol = gemm_tolerance(y, s, True)
+    bad = np.argwhere(np.abs(got - y) > tol)
+    assert bad.size == 0, "%d of %d out of tolerance" % (len(bad), got.size)
+
+
+def test_gemm_lora_host_validation():
+    """Host-side rules of nvfp4_gemm_lora (nothing is launched)."""
+    from nvfp4_block_scaled_20_b200 import capi
+    p = 1 << 12
+    args = lambda rank, ldu, scale, scr: (p, p, p, p, p, p, 128, 128, 256, p, ldu, p, rank, rank,  # noqa: E731
+                                          scale, scr, 1 << 20, p, 0, 128, 0, p, 4096, None)
+    assert capi.nvfp4_gemm_lora(*args(96, 96, 1.0, p)) == 2        # rank not a multiple of 64
+    assert capi.nvfp4_gemm_lora(*args(128, 100, 1.0, p)) == 2      # ldu < rank... (100 < 128)
+    assert capi.nvfp4_gemm_lora(*args(128, 128, float("inf"), p)) == 1
+    assert capi.nvfp4_gemm_lora(*args(128, 128, 1.0, p + 8)) == 3  # scratch misaligned
+    assert capi.nvfp4_lora_scratch_bytes(2640, 128) == 2640 * 128 * 4
