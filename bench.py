@@ -411,6 +411,9 @@ def main():
     ap.add_argument("--rows", default="auto", choices=["auto", "on", "off"],
                     help="also time every hot-path row at its full workload size "
                          "(auto: on a single GPU only)")
+    ap.add_argument("--profiler-range", action="store_true",
+                    help="bracket the timed step replays with cudaProfilerStart/Stop (for a "
+                         "launch list taken with ncu --profile-from-start off)")
     ap.add_argument("--profile", default=None, choices=sorted(PROFILE_CASES),
                     help="run one case a few times (untimed, no JSON line): the program "
                          "the ncu captures under profiles/ are taken on")
@@ -516,8 +519,12 @@ def main():
     time.sleep(0.2)
     barrier(world)
     torch.cuda.synchronize(dev)
+    if args.profiler_range:
+        torch.cuda.profiler.start()
     step_ms = timed(graphs["step"], args.steps)
     torch.cuda.synchronize(dev)
+    if args.profiler_range:
+        torch.cuda.profiler.stop()
     barrier(world)
     # per-kernel breakdown (same protocol)
     reps = max(10, min(args.steps, 100))
