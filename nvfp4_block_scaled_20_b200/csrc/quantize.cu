@@ -90,10 +90,22 @@ struct Slice {
 // the HBM latency at three CTAs per SM; the load form itself was measured not
 // to matter: non-coherent, plain, evict-first and bulk copies stream alike).
 constexpr int kAmaxDepth = 8;
+// Address of 16-block u of a row-major tensor: contiguous rows (ld == cols)
+// need no division; otherwise the row comes from a multiply-high division.
+template <typename T>
+__device__ __forceinline__ const T* block_ptr(const T* x, uint64_t u, bool contig, uint32_t kbpr,
+                                              FastDiv div, int64_t ld) {
+  if (contig) return x + u * 16;
+  const uint32_t r = fastdiv((uint32_t)u, div);
+  return x + (int64_t)r * ld + (int64_t)((uint32_t)u - r * kbpr) * 16;
+}
+
 __device__ float amax_rows_bf16_raw(const QTensor& q, const Slice sl) {
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(q.x);
   const uint32_t kbpr = (uint32_t)(q.cols >> 4);
   const uint64_t nblk = (uint64_t)q.rows * kbpr;
+  const bool contig = q.ld == q.cols;
+  const FastDiv div = make_fastdiv(kbpr);
   const uint64_t stride = (uint64_t)sl.ncta * kThreads;
   uint32_t m2 = 0u;
   for (uint64_t u = (uint64_t)sl.cta * kThreads + threadIdx.x; u < nblk; u += kAmaxDepth * stride) {
@@ -102,8 +114,7 @@ __device__ float amax_rows_bf16_raw(const QTensor& q, const Slice sl) {
     for (int j = 0; j < kAmaxDepth; ++j) {
       const uint64_t uj = u + j * stride;
       if (uj < nblk) {
-        const uint32_t r = (uint32_t)uj / kbpr, kb = (uint32_t)uj - r * kbpr;
-        load16_raw(x + (int64_t)r * q.ld + (int64_t)kb * 16, w[j]);
+        load16_raw(block_ptr(x, uj, contig, kbpr, div, q.ld), w[j]);
       } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) w[j][i] = 0u;
@@ -123,6 +134,8 @@ __device__ float amax_rows(const QTensor& q, uint32_t mask, const Slice sl) {
   const T* x = static_cast<const T*>(q.x);
   const uint32_t kbpr = (uint32_t)(q.cols >> 4);
   const uint64_t nblk = (uint64_t)q.rows * kbpr;
+  const bool contig = q.ld == q.cols;
+  const FastDiv div = make_fastdiv(kbpr);
   const uint64_t stride = (uint64_t)sl.ncta * kThreads;
   float m = 0.0f;
   // two blocks per thread per trip, both loads issued before any use
@@ -132,8 +145,7 @@ __device__ float amax_rows(const QTensor& q, uint32_t mask, const Slice sl) {
     for (int j = 0; j < 2; ++j) {
       const uint64_t uj = u + j * stride;
       if (uj < nblk) {
-        const uint32_t r = (uint32_t)uj / kbpr, kb = (uint32_t)uj - r * kbpr;
-        load16(x + (int64_t)r * q.ld + (int64_t)kb * 16, v[j]);
+        load16(block_ptr(x, uj, contig, kbpr, div, q.ld), v[j]);
       } else {
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[j][i] = 0.0f;
@@ -358,17 +370,15 @@ __device__ void encode_rows(const QTensor& q, float alpha, const QBatch& p, uint
   const bool fos = p.four_over_six != 0;
   const ScaleCtx ctx = make_scale_ctx(alpha);
   const uint32_t stride = sl.ncta * kThreads;
-  auto src = [&](uint32_t b) {
-    const uint32_t r = fastdiv(b, div);
-    return x + (int64_t)r * q.ld + (int64_t)(b - r * kbpr) * 16;
-  };
-  auto codes_at = [&](uint32_t b) {
-    const uint32_t r = fastdiv(b, div);
-    return q.codes + (int64_t)r * (q.cols >> 1) + (int64_t)(b - r * kbpr) * 8;
-  };
+  // codes rows are cols / 2 bytes, so block b's codes start at 8 b; a
+  // contiguous input (ld == cols) and row-major scales need no division
+  const bool contig = q.ld == q.cols;
+  auto src = [&](uint32_t b) { return block_ptr(x, b, contig, kbpr, div, q.ld); };
+  auto codes_at = [&](uint32_t b) { return q.codes + (int64_t)b * 8; };
   auto scale_at = [&](uint32_t b) {
+    if (p.sf_layout == 0) return q.scales + b;
     const uint32_t r = fastdiv(b, div);
-    return q.scales + sf_offset(r, b - r * kbpr, kbpr, p.sf_layout);
+    return q.scales + sf_offset(r, b - r * kbpr, kbpr, 1);
   };
   // bf16 blocks are queued with their raw input, fp32 blocks are reloaded
   constexpr bool kCarry = std::is_same<T, __nv_bfloat16>::value;
@@ -499,8 +509,22 @@ __device__ void encode_cols(const QTensor& q, float alpha, const QBatch& p, uint
 // (bounded) and stops.
 constexpr int kTmaRows = 64, kTmaCols = 128;
 constexpr int kTmaTileBytes = kTmaRows * kTmaCols * 2;
+// tiles in flight per CTA: the amax pass, the encode pass (which also holds
+// its queue of handed-back blocks in shared memory, kColsQueueCap entries per
+// warp) and the CTAs per SM the encode pass is compiled for
 constexpr int kTmaStages = 4;
-constexpr int kTmaSmemBytes = kTmaStages * kTmaTileBytes + 128;
+#ifndef NVFP4_COLS_ENC_STAGES
+#define NVFP4_COLS_ENC_STAGES 4
+#endif
+#ifndef NVFP4_COLS_QCAP
+#define NVFP4_COLS_QCAP 128
+#endif
+#ifndef NVFP4_COLS_MINB
+#define NVFP4_COLS_MINB 2
+#endif
+constexpr int kColsEncStages = NVFP4_COLS_ENC_STAGES;
+constexpr int kColsQueueCap = NVFP4_COLS_QCAP;
+constexpr int tma_smem_bytes(int stages) { return stages * kTmaTileBytes + 128; }
 constexpr uint64_t kTmaWaitNs = 2000000000ull, kTmaDrainNs = 200000000ull;
 
 struct ColsMaps {
@@ -537,7 +561,7 @@ __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, uint64_t
 // CTA = sl.cta + i * sl.ncta): thread 0 keeps the next kTmaStages - 1 tiles
 // loading; fn(tile, smem of the tile) runs on every thread.  Returns false
 // after a wait ran out (error recorded, loads in flight drained).
-template <typename F>
+template <int kTmaStages, typename F>
 __device__ bool tma_tile_loop(const CUtensorMap* map, const QTensor& q, const Slice sl,
                               uint8_t* smem, uint32_t* err, F&& fn) {
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTmaStages * kTmaTileBytes);
@@ -622,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 3)
   const QTensor& q = p.t[t];
   const Slice sl{blockIdx.x, gridDim.x};
   float m = 0.0f;
-  tma_tile_loop(&maps.m[t], q, sl, smem, p.err, [&](uint32_t, const uint8_t* tile) {
+  tma_tile_loop<kTmaStages>(&maps.m[t], q, sl, smem, p.err, [&](uint32_t, const uint8_t* tile) {
     uint32_t w[16];
     tile_words<RHT>(tile, p.mask, w);  // zero past the tensor's edges: no effect on the max
 #pragma unroll
@@ -638,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 3)
 }
 
 template <bool RHT>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, NVFP4_COLS_MINB)
     encode_cols_tma_kernel(const __grid_constant__ QBatch p, const __grid_constant__ ColsMaps maps,
                            int ga) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -656,8 +680,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   // per-warp queue of handed-back blocks; each entry carries the block's 16
   // input values (bf16, element j in half j % 2 of word j / 2), so the redo
   // reads shared memory, not the tile's rows in global memory again
-  __shared__ uint2 queue[kThreads / 32][kQueueCap];
-  __shared__ uint4 qdata[kThreads / 32][kQueueCap][2];
+  __shared__ uint2 queue[kThreads / 32][kColsQueueCap];
+  __shared__ uint4 qdata[kThreads / 32][kColsQueueCap][2];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint32_t qn = 0;  // same value on every lane
   const uint32_t kb_total = (uint32_t)(q.rows >> 4);
@@ -687,7 +711,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncwarp();
     qn = 0;
   };
-  tma_tile_loop(&maps.m[t], q, sl, smem, p.err, [&](uint32_t tile_id, const uint8_t* tile) {
+  tma_tile_loop<kColsEncStages>(&maps.m[t], q, sl, smem, p.err,
+                                [&](uint32_t tile_id, const uint8_t* tile) {
     uint32_t w[16];
     tile_words<RHT>(tile, p.mask, w);
     const uint32_t kb = (tile_id / ntc) * (kTmaRows / 16) + (threadIdx.x >> 6);
@@ -723,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       qn += __popc(m);
     }
-    if (qn > kQueueCap - 64) drain();
+    if (qn > kColsQueueCap - 64) drain();
   });
   drain();
   if (p.sf_layout == 1) zero_sf_padding(q.scales, q.cols, kb_total, sl);
@@ -1032,61 +1057,79 @@ __global__ void __launch_bounds__(kThreads) dequant_rows_kernel(const __grid_con
 
 // ------------------------------------------------------------------------
 // Transpose of a 2D (16x16-tile) encoding: the data-gradient GEMM's weight
-// operand.  A CTA moves 64 rows x 256 codes through shared memory (one byte
-// per code; rows padded to 260 bytes): each thread loads 64 codes of one row
-// (four 8-byte loads in flight), then four threads write each output row's
-// 32 contiguous bytes;
-// each output block's scale comes from its tile: output (c, b) takes input
-// (16 b, c / 16).  rows and cols are multiples of 16.
+// operand.  A CTA takes 64 input rows x 256 input columns of codes.  Thread
+// (i, j) = (t / 32, t % 32) loads the 8 x 8 block of codes at rows
+// 8 i .. 8 i + 7, columns 8 j .. 8 j + 7 as eight 32-bit words (a warp reads
+// 128 contiguous bytes of one row per load) and transposes it in registers:
+// three stages swap 4x4, 2x2 and 1x1 blocks of 4-bit codes with masks and
+// shifts, after which word k holds input column 8 j + k with the code of
+// input row 8 i + r in nibble r.  The words go through shared memory, and
+// four threads write each output row (input column) of the tile: thread q of
+// the four writes the 8 bytes of input rows 16 q .. 16 q + 15 and the scale
+// byte of that 16 x 16 tile (output block (c, b) takes the tile scale of
+// input (16 b, c / 16)), so a warp store covers whole 32-byte sectors of
+// eight output rows.  The shared-memory word of (staging row k, output row o)
+// sits at column tr_slot(o, k), which keeps both sides free of bank
+// conflicts.  rows and cols are multiples of 16.
 constexpr int kTrRows = 64, kTrCols = 256;
+__device__ __forceinline__ void nib_swap(uint32_t& a, uint32_t& b, int s, uint32_t m) {
+  const uint32_t t = ((a >> s) ^ b) & m;
+  a ^= t << s;
+  b ^= t;
+}
+__device__ __forceinline__ int tr_slot(int o, int k) {
+  const int j = o >> 3;
+  return 8 * j + (((o & 7) + j + (j >> 3) + k) & 7);
+}
 __global__ void __launch_bounds__(kThreads)
     transpose_2d_kernel(const uint8_t* codes, const uint8_t* scales, int sf_in, int64_t rows,
                         int64_t cols, uint8_t* out_codes, uint8_t* out_scales, int sf_out) {
-  __shared__ __align__(16) uint8_t t[kTrRows][kTrCols + 4];
+  __shared__ uint32_t t[8][kTrCols];  // [input row block][output row, swizzled]
   const int64_t tiles_c = (cols + kTrCols - 1) / kTrCols;
   const int64_t ntiles = ((rows + kTrRows - 1) / kTrRows) * tiles_c;
-  const int lr = threadIdx.x >> 2, part = threadIdx.x & 3;
+  const int i = threadIdx.x >> 5, j = threadIdx.x & 31;
+  // write side: per pass of 64 output rows, warp i takes two rows from each
+  // of four row groups of eight, so that its 32 reads hit 32 banks
+  const int q = j & 3, e = j >> 2;
+  const int o_lo = 8 * (4 * (i & 1) + (e & 3)) + 2 * (i >> 1) + (e >> 2);
+  const int64_t in_row_bytes = cols >> 1, out_row_bytes = rows >> 1;
+  const int64_t kb_out = rows >> 4, kb_in = cols >> 4;
   for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
     const int64_t r0 = (tile / tiles_c) * kTrRows, c0 = (tile % tiles_c) * kTrCols;
-    {  // thread: row r0 + lr, codes c0 + 64 part .. + 63 (four 16-code chunks)
-      const int64_t r = r0 + lr;
-      uint2 w[4];
+    {
+      uint32_t w[8];
+      const int64_t r = r0 + 8 * i, c = c0 + 8 * j;
+      const uint8_t* src = codes + r * in_row_bytes + (c >> 1);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int64_t c = c0 + 64 * part + 16 * j;
-        w[j] = (r < rows && c < cols)
-                   ? __ldg(reinterpret_cast<const uint2*>(codes + r * (cols >> 1) + (c >> 1)))
-                   : make_uint2(0u, 0u);
-      }
-      uint32_t* dst = reinterpret_cast<uint32_t*>(&t[lr][64 * part]);
+      for (int k = 0; k < 8; ++k)
+        w[k] = (r + k < rows && c < cols) ? __ldg(reinterpret_cast<const uint32_t*>(
+                                                src + (int64_t)k * in_row_bytes))
+                                          : 0u;
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+      for (int k = 0; k < 4; ++k) nib_swap(w[k], w[k + 4], 16, 0x0000FFFFu);
+      nib_swap(w[0], w[2], 8, 0x00FF00FFu);
+      nib_swap(w[1], w[3], 8, 0x00FF00FFu);
+      nib_swap(w[4], w[6], 8, 0x00FF00FFu);
+      nib_swap(w[5], w[7], 8, 0x00FF00FFu);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t v = h ? w[j].y : w[j].x;  // 8 codes, code i in bits 4i..4i+3
-          dst[4 * j + 2 * h] = (v & 0xFu) | ((v >> 4) & 0xFu) << 8 | ((v >> 8) & 0xFu) << 16 |
-                               ((v >> 12) & 0xFu) << 24;
-          dst[4 * j + 2 * h + 1] = ((v >> 16) & 0xFu) | ((v >> 20) & 0xFu) << 8 |
-                                   ((v >> 24) & 0xFu) << 16 | (v >> 28) << 24;
-        }
+      for (int k = 0; k < 8; k += 2) nib_swap(w[k], w[k + 1], 4, 0x0F0F0F0Fu);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) t[i][tr_slot(8 * j + k, i)] = w[k];
     }
     __syncthreads();
-    // output rows c0 .. c0 + 255 (input columns) in four passes of 64; the
-    // four threads of an output row write its 32 contiguous bytes
-#pragma unroll 1
-    for (int pass = 0; pass < kTrCols / 64; ++pass) {
-      const int lc = pass * 64 + lr, j = part;
-      const int64_t c = c0 + lc, r = r0 + 16 * j;
-      if (c < cols && r < rows) {
-        uint32_t lo = 0u, hi = 0u;
+    // 16 input rows = 8 bytes = 2 words; rows - r0 is a multiple of 16
+    if (16 * q < rows - r0) {
+      const int64_t rb = (r0 >> 4) + q;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          lo |= (uint32_t)t[16 * j + i][lc] << (4 * i);
-          hi |= (uint32_t)t[16 * j + 8 + i][lc] << (4 * i);
+      for (int pass = 0; pass < kTrCols / 64; ++pass) {
+        const int o = 64 * pass + o_lo;
+        const int64_t c = c0 + o;
+        if (c < cols) {
+          *reinterpret_cast<uint2*>(out_codes + c * out_row_bytes + (r0 >> 1) + 8 * q) =
+              make_uint2(t[2 * q][tr_slot(o, 2 * q)], t[2 * q + 1][tr_slot(o, 2 * q + 1)]);
+          out_scales[sf_offset(c, rb, kb_out, sf_out)] =
+              __ldg(scales + sf_offset(rb * 16, c >> 4, kb_in, sf_in));
         }
-        *reinterpret_cast<uint2*>(out_codes + c * (rows >> 1) + (r >> 1)) = make_uint2(lo, hi);
-        out_scales[sf_offset(c, r >> 4, rows >> 4, sf_out)] =
-            __ldg(scales + sf_offset(r, c >> 4, cols >> 4, sf_in));
       }
     }
     __syncthreads();
@@ -1220,11 +1263,11 @@ bool make_cols_maps(const QBatch& b, ColsMaps& maps) {
 
 template <typename K>
 cudaError_t launch_maps(K kern, dim3 grid, cudaStream_t s, bool pdl, const QBatch& b,
-                        const ColsMaps& maps, int ga, bool with_ga) {
+                        const ColsMaps& maps, int ga, bool with_ga, int smem_bytes) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kTmaSmemBytes;
+  cfg.dynamicSmemBytes = smem_bytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1244,10 +1287,10 @@ cudaError_t launch_cols_tma(const QBatch& b, cudaStream_t s) {
   static const bool attrs_ok = [] {
     return cudaFuncSetAttribute(amax_cols_tma_kernel<RHT>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                kTmaSmemBytes) == cudaSuccess &&
+                                tma_smem_bytes(kTmaStages)) == cudaSuccess &&
            cudaFuncSetAttribute(encode_cols_tma_kernel<RHT>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                kTmaSmemBytes) == cudaSuccess;
+                                tma_smem_bytes(kColsEncStages)) == cudaSuccess;
   }();
   if (!attrs_ok) return cudaErrorNotSupported;
   uint64_t tiles = 0;
@@ -1263,14 +1306,16 @@ cudaError_t launch_cols_tma(const QBatch& b, cudaStream_t s) {
     if (cap > (uint64_t)kMaxAmaxCtas) cap = kMaxAmaxCtas;
     if (cap < 1) cap = 1;
     ga = (int)(tiles < cap ? (tiles < 1 ? 1 : tiles) : cap);
-    cudaError_t e = launch_maps(amax_cols_tma_kernel<RHT>, dim3(ga, b.n), s, false, b, maps, 0, false);
+    cudaError_t e = launch_maps(amax_cols_tma_kernel<RHT>, dim3(ga, b.n), s, false, b, maps, 0,
+                                false, tma_smem_bytes(kTmaStages));
     if (e != cudaSuccess) return e;
     if (b.amax_only) return launch_ex(finalize_kernel, dim3(b.n), s, true, b, ga);
   }
-  uint64_t cap = (uint64_t)num_sms() * 2 / (uint64_t)b.n;
+  uint64_t cap = (uint64_t)num_sms() * NVFP4_COLS_MINB / (uint64_t)b.n;
   if (cap < 1) cap = 1;
   const unsigned gx = (unsigned)(tiles < cap ? (tiles < 1 ? 1 : tiles) : cap);
-  return launch_maps(encode_cols_tma_kernel<RHT>, dim3(gx, b.n), s, !b.gs_in, b, maps, ga, true);
+  return launch_maps(encode_cols_tma_kernel<RHT>, dim3(gx, b.n), s, !b.gs_in, b, maps, ga, true,
+                     tma_smem_bytes(kColsEncStages));
 }
 
 template <typename T>
