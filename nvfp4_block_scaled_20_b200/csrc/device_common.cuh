@@ -713,11 +713,15 @@ __device__ __forceinline__ uint32_t quantize_block16_pairs(const uint64_t yy[8],
 }
 
 // Byte offset of scale (r, kb) in the chosen layout.
+// Every tensor the library encodes has fewer than 2^32 blocks (the entry
+// points check), so rows, block columns and the 512-byte atom index all fit in
+// 32 bits; only the final byte offset is widened.
 __device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t kb, int64_t kb_total, int layout) {
-  if (layout == 0) return r * kb_total + kb;
-  const int64_t kb_groups = (kb_total + 3) >> 2;
-  return (((r >> 7) * kb_groups + (kb >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) +
-         (kb & 3);
+  const uint32_t r32 = (uint32_t)r, kb32 = (uint32_t)kb, kt = (uint32_t)kb_total;
+  if (layout == 0) return (int64_t)((uint64_t)r32 * kt + kb32);
+  const uint32_t groups = (kt + 3) >> 2;
+  return (int64_t)(((uint64_t)((r32 >> 7) * groups + (kb32 >> 2)) << 9) +
+                   (((r32 & 31) << 4) | (((r32 >> 5) & 3) << 2) | (kb32 & 3)));
 }
 
 // Atomic max of a non-negative float stored as its bit pattern.

@@ -350,18 +350,22 @@ __host__ __device__ constexpr uint32_t instr_desc_bf16(int M, int N) {
 
 // GELU(tanh form) in fp32: 0.5 y (1 + tanh(u)), u = sqrt(2/pi) (y + 0.044715
 // y^3), evaluated as y * sigmoid(2u) = y / (1 + exp(-2u)) (the same function:
-// 1 + tanh(u) = 2 / (1 + exp(-2u))), with the __expf / __fdividef intrinsics.
-// For |2u| up to the point where the quotient saturates, their relative
-// errors (a few ulp of exp, growing with |2u|, and 2 ulp of the quotient) move
-// the result by less than 2^-18 |y|; exp(-2u) overflowing to +inf gives
-// -0 (GELU of a large negative y is below any fp32 of its magnitude's
-// scale), and __fdividef returning 0 for denominators above 2^126 does the
-// same.  So |GELU_gpu(y) - GELU(y)| < 2^-17 |y| -- negligible against the
-// GEMM's 1e-3 sum_k |a_k b_k|.
+// 1 + tanh(u) = 2 / (1 + exp(-2u))), with exp(-2u) = 2^(y (c0 + c1 y^2)),
+// c0 = -2 log2(e) sqrt(2/pi), c1 = 0.044715 c0, through the hardware ex2 and
+// the __fdividef intrinsic.  For |2u| up to the point where the quotient
+// saturates, the relative errors (the exponent's few ulp, scaled by its
+// magnitude, a couple of ulp of ex2 and of the quotient) move the result by
+// less than 2^-18 |y|; 2^(...) overflowing to +inf gives -0 (GELU of a large
+// negative y is below any fp32 of its magnitude's scale), and __fdividef
+// returning 0 for denominators above 2^126 does the same.  So
+// |GELU_gpu(y) - GELU(y)| < 2^-17 |y| -- negligible against the GEMM's
+// 1e-3 sum_k |a_k b_k|.
 __device__ __forceinline__ float gelu_tanh(float y) {
-  const float k0 = 0.7978845608028654f, k01 = 0.7978845608028654f * 0.044715f;
-  const float inner = y * fmaf(k01, y * y, k0);
-  return __fdividef(y, 1.0f + __expf(-2.0f * inner));
+  constexpr double kC0 = -2.0 * 1.4426950408889634 * 0.7978845608028654;
+  const float c0 = (float)kC0, c1 = (float)(kC0 * 0.044715);
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(y * fmaf(c1, y * y, c0)));
+  return __fdividef(y, 1.0f + e);
 }
 
 struct Params {

@@ -1057,7 +1057,8 @@ __global__ void __launch_bounds__(kThreads) dequant_rows_kernel(const __grid_con
 
 // ------------------------------------------------------------------------
 // Transpose of a 2D (16x16-tile) encoding: the data-gradient GEMM's weight
-// operand.  A CTA takes 64 input rows x 256 input columns of codes.  Thread
+// operand.  A CTA takes 64 input rows x 256 input columns of codes, and loads
+// the next tile's codes and scale bytes while it writes the current one.  Thread
 // (i, j) = (t / 32, t % 32) loads the 8 x 8 block of codes at rows
 // 8 i .. 8 i + 7, columns 8 j .. 8 j + 7 as eight 32-bit words (a warp reads
 // 128 contiguous bytes of one row per load) and transposes it in registers:
@@ -1085,50 +1086,70 @@ __global__ void __launch_bounds__(kThreads)
     transpose_2d_kernel(const uint8_t* codes, const uint8_t* scales, int sf_in, int64_t rows,
                         int64_t cols, uint8_t* out_codes, uint8_t* out_scales, int sf_out) {
   __shared__ uint32_t t[8][kTrCols];  // [input row block][output row, swizzled]
-  const int64_t tiles_c = (cols + kTrCols - 1) / kTrCols;
-  const int64_t ntiles = ((rows + kTrRows - 1) / kTrRows) * tiles_c;
+  const uint32_t tiles_c = (uint32_t)((cols + kTrCols - 1) / kTrCols);
+  const uint32_t ntiles = (uint32_t)((rows + kTrRows - 1) / kTrRows) * tiles_c;
   const int i = threadIdx.x >> 5, j = threadIdx.x & 31;
   // write side: per pass of 64 output rows, warp i takes two rows from each
   // of four row groups of eight, so that its 32 reads hit 32 banks
   const int q = j & 3, e = j >> 2;
   const int o_lo = 8 * (4 * (i & 1) + (e & 3)) + 2 * (i >> 1) + (e >> 2);
   const int64_t in_row_bytes = cols >> 1, out_row_bytes = rows >> 1;
-  const int64_t kb_out = rows >> 4, kb_in = cols >> 4;
-  for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-    const int64_t r0 = (tile / tiles_c) * kTrRows, c0 = (tile % tiles_c) * kTrCols;
-    {
-      uint32_t w[8];
-      const int64_t r = r0 + 8 * i, c = c0 + 8 * j;
-      const uint8_t* src = codes + r * in_row_bytes + (c >> 1);
+  const uint32_t kb_out = (uint32_t)(rows >> 4), kb_in = (uint32_t)(cols >> 4);
+  constexpr int kPasses = kTrCols / 64;
+  // A tile's global reads, issued one tile ahead: the thread's 8 x 8 block of
+  // codes and the scale bytes of the output blocks it writes.
+  uint32_t w[8], sc[kPasses];
+  auto fetch = [&](uint32_t tile) {
+    const uint32_t tr = tile / tiles_c;
+    const int64_t r0 = (int64_t)tr * kTrRows, c0 = (int64_t)(tile - tr * tiles_c) * kTrCols;
+    const int64_t r = r0 + 8 * i, c = c0 + 8 * j;
+    const uint8_t* src = codes + r * in_row_bytes + (c >> 1);
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
-        w[k] = (r + k < rows && c < cols) ? __ldg(reinterpret_cast<const uint32_t*>(
-                                                src + (int64_t)k * in_row_bytes))
-                                          : 0u;
+    for (int k = 0; k < 8; ++k)
+      w[k] = (r + k < rows && c < cols)
+                 ? __ldg(reinterpret_cast<const uint32_t*>(src + (int64_t)k * in_row_bytes))
+                 : 0u;
+    const bool rows_in = 16 * q < rows - r0;
+    const uint32_t rb16 = (uint32_t)(r0 + 16 * q);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) nib_swap(w[k], w[k + 4], 16, 0x0000FFFFu);
-      nib_swap(w[0], w[2], 8, 0x00FF00FFu);
-      nib_swap(w[1], w[3], 8, 0x00FF00FFu);
-      nib_swap(w[4], w[6], 8, 0x00FF00FFu);
-      nib_swap(w[5], w[7], 8, 0x00FF00FFu);
-#pragma unroll
-      for (int k = 0; k < 8; k += 2) nib_swap(w[k], w[k + 1], 4, 0x0F0F0F0Fu);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) t[i][tr_slot(8 * j + k, i)] = w[k];
+    for (int pass = 0; pass < kPasses; ++pass) {
+      const int64_t cc = c0 + 64 * pass + o_lo;
+      sc[pass] = (rows_in && cc < cols)
+                     ? (uint32_t)__ldg(scales + sf_offset(rb16, (uint32_t)(cc >> 4), kb_in, sf_in))
+                     : 0u;
     }
+  };
+  if (blockIdx.x < ntiles) fetch(blockIdx.x);
+  for (uint32_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const uint32_t tr = tile / tiles_c;
+    const int64_t r0 = (int64_t)tr * kTrRows, c0 = (int64_t)(tile - tr * tiles_c) * kTrCols;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) nib_swap(w[k], w[k + 4], 16, 0x0000FFFFu);
+    nib_swap(w[0], w[2], 8, 0x00FF00FFu);
+    nib_swap(w[1], w[3], 8, 0x00FF00FFu);
+    nib_swap(w[4], w[6], 8, 0x00FF00FFu);
+    nib_swap(w[5], w[7], 8, 0x00FF00FFu);
+#pragma unroll
+    for (int k = 0; k < 8; k += 2) nib_swap(w[k], w[k + 1], 4, 0x0F0F0F0Fu);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t[i][tr_slot(8 * j + k, i)] = w[k];
+    uint32_t s_cur[kPasses];
+#pragma unroll
+    for (int pass = 0; pass < kPasses; ++pass) s_cur[pass] = sc[pass];
     __syncthreads();
+    if (tile + gridDim.x < ntiles) fetch(tile + gridDim.x);  // in flight during the writes
     // 16 input rows = 8 bytes = 2 words; rows - r0 is a multiple of 16
     if (16 * q < rows - r0) {
-      const int64_t rb = (r0 >> 4) + q;
+      const uint32_t rb = (uint32_t)(r0 >> 4) + (uint32_t)q;
+      uint8_t* dst = out_codes + (r0 >> 1) + 8 * q;
 #pragma unroll
-      for (int pass = 0; pass < kTrCols / 64; ++pass) {
+      for (int pass = 0; pass < kPasses; ++pass) {
         const int o = 64 * pass + o_lo;
         const int64_t c = c0 + o;
         if (c < cols) {
-          *reinterpret_cast<uint2*>(out_codes + c * out_row_bytes + (r0 >> 1) + 8 * q) =
+          *reinterpret_cast<uint2*>(dst + c * out_row_bytes) =
               make_uint2(t[2 * q][tr_slot(o, 2 * q)], t[2 * q + 1][tr_slot(o, 2 * q + 1)]);
-          out_scales[sf_offset(c, rb, kb_out, sf_out)] =
-              __ldg(scales + sf_offset(rb * 16, c >> 4, kb_in, sf_in));
+          out_scales[sf_offset((uint32_t)c, rb, kb_out, sf_out)] = (uint8_t)s_cur[pass];
         }
       }
     }
@@ -1427,7 +1448,17 @@ cudaError_t launch_transpose_2d(const uint8_t* codes, const uint8_t* scales, int
                                 uint8_t* out_scales, int sf_out, cudaStream_t s) {
   const uint64_t tiles = (uint64_t)((rows + kTrRows - 1) / kTrRows) *
                          (uint64_t)((cols + kTrCols - 1) / kTrCols);
-  const uint64_t cap = (uint64_t)num_sms() * 8;
+  // one wave of resident CTAs, each looping over tiles (its next tile's loads
+  // overlap its current tile's stores)
+  static const int per_sm = [] {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, transpose_2d_kernel, kThreads, 0) !=
+            cudaSuccess ||
+        n < 1)
+      n = 4;
+    return n;
+  }();
+  const uint64_t cap = (uint64_t)num_sms() * (uint64_t)per_sm;
   const int grid = (int)(tiles < cap ? (tiles < 1 ? 1 : tiles) : cap);
   transpose_2d_kernel<<<grid, kThreads, 0, s>>>(codes, scales, sf_in, rows, cols, out_codes,
                                                out_scales, sf_out);
