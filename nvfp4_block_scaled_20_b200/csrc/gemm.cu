@@ -609,7 +609,14 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (leader && lane == 0) {
       constexpr uint32_t idesc = instr_desc(2 * BM, BN);
+      static_assert(kSfSlots == 2, "the issue loop alternates two scale slots");
       uint32_t it = 0, tile_i = 0;
+      // ring position of stage `it` and the phase parities it waits for,
+      // advanced incrementally (no division in the issue loop)
+      uint32_t st = 0, st_ph = 0, slot = 0, slot_ph = 0;
+      const uint64_t desc_a0 = operand_desc(smem_u32(sA)), desc_b0 = operand_desc(smem_u32(sB));
+      const uint32_t t_sf0 = tmem + kSfSlotCol, t_sf1 = tmem + kSfSlotCol + kSfSlotCols;
+      const int nmma_last = (p.K - (num_kt - 1) * BK) / MMA_K;
       bool ok = true;
       // test hook (nvfp4_set_test_stall): a wait that runs out after the
       // pipeline bound while the producers' first stages are in flight
@@ -629,32 +636,41 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         tc_fence_after();
         const uint32_t t_acc = tmem + (b ? kAcc1Col : 0u);
         for (int kt = 0; kt < total_kt; ++kt, ++it) {
-          const int s = it % kStages;
-          const uint32_t slot = it % kSfSlots;
-          if (!mbar_wait(smem_u32(&full[s]), (it / kStages) & 1u, abort_flag, p.wait_limit_ns) ||
-              !mbar_wait(smem_u32(&sf_full[slot]), (it / kSfSlots) & 1u, abort_flag, p.wait_limit_ns)) {
+          if (!mbar_wait(smem_u32(&full[st]), st_ph, abort_flag, p.wait_limit_ns) ||
+              !mbar_wait(smem_u32(&sf_full[slot]), slot_ph, abort_flag, p.wait_limit_ns)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(sA + s * kABytes);
-          const uint32_t b_base = smem_u32(sB + s * kBBytes);
+          // descriptors of this stage's tiles: the start-address field (bits
+          // 0-13, address / 16) advances by the stage offset and by 32 bytes
+          // (2 units) per MMA k-block; shared memory is below 256 KB, so the
+          // field never carries into the next one
+          const uint64_t da = desc_a0 + (uint64_t)(st * (kABytes >> 4));
+          const uint64_t db = desc_b0 + (uint64_t)(st * (kBBytes >> 4));
           if (kt >= num_kt) {
             // LoRA stage: four bf16 MMAs (K = 16, 32 bytes of each row) into the
             // same accumulator, which the FP4 stages have initialised
             constexpr uint32_t idesc16 = instr_desc_bf16(2 * BM, BN);
-            for (int k = 0; k < 4; ++k)
-              tc_mma_pair_bf16(t_acc, operand_desc(a_base + 32 * k), operand_desc(b_base + 32 * k),
-                               idesc16, 1u);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) tc_mma_pair_bf16(t_acc, da + 2 * k, db + 2 * k, idesc16, 1u);
           } else {
-            const int nmma = min(4, (p.K - kt * BK) / MMA_K);
-            const uint32_t t_sf = tmem + kSfSlotCol + slot * kSfSlotCols;
-            for (int k = 0; k < nmma; ++k)
-              tc_mma_pair(t_acc, operand_desc(a_base + 32 * k), operand_desc(b_base + 32 * k),
-                          idesc, t_sf + 4 * k, t_sf + 16 + 8 * k, (kt > 0 || k > 0) ? 1u : 0u);
+            const int nmma = kt == num_kt - 1 ? nmma_last : 4;
+            const uint32_t t_sf = slot ? t_sf1 : t_sf0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              if (k < nmma)
+                tc_mma_pair(t_acc, da + 2 * k, db + 2 * k, idesc, t_sf + 4 * k, t_sf + 16 + 8 * k,
+                            (kt > 0 || k > 0) ? 1u : 0u);
           }
-          tc_commit_pair(smem_u32(&empty[s]));
+          tc_commit_pair(smem_u32(&empty[st]));
           tc_commit_pair(smem_u32(&sf_empty[slot]));
+          if (++st == kStages) {
+            st = 0;
+            st_ph ^= 1u;
+          }
+          slot ^= 1u;
+          slot_ph ^= slot == 0u ? 1u : 0u;
         }
         // signals both CTAs once this tile's MMAs (and everything before) completed
         tc_commit_pair(smem_u32(&acc_full[b]));
