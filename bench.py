@@ -44,7 +44,16 @@ QOUT = 0.5 + 1.0 / 16  # bytes written per quantized element (codes + scale byte
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch of
 # the step's kernels from ncu captures, valid only for the sources they were
 # taken on (hash of the kernel's source files).
-TRAFFIC = {}
+TRAFFIC = {
+    # one ncu capture of the full-size step: python bench.py --profile
+    # wgrad_step, the first rep's five launches (after the four setup ones)
+    "gemm": {"bytes_per_launch": 867592960 + 156140800,
+             "source_sha256": "8e9e134b290f2562be354aa170c830daca15e84b1f45f6452bf99e03ed875a35"},
+    "encode_x": {"bytes_per_launch": 953817600 + 251720448,
+                 "source_sha256": "9934fb8729244c8bf3bcd7f71c02b47b032a710e8124a3f1052c3f65c591eec7"},
+    "amax_x": {"bytes_per_launch": 939637760 + 723968,
+               "source_sha256": "9934fb8729244c8bf3bcd7f71c02b47b032a710e8124a3f1052c3f65c591eec7"},
+}
 
 
 def _sources_digest(files):
