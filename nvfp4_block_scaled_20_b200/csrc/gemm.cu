@@ -466,8 +466,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   uint64_t* sf_in = full + kStages;           // [kStages] this CTA's scale atoms landed
   uint64_t* empty = sf_in + kStages;          // [kStages] stage free: MMAs done + scales read
   uint64_t* sf_full = empty + kStages;        // [2] scale slot written by both CTAs (leader)
-  uint64_t* sf_empty = sf_full + kSfSlots;    // [2] scale slot's MMAs done
-  uint64_t* acc_full = sf_empty + kSfSlots;   // [2] accumulator complete
+  uint64_t* acc_full = sf_full + kSfSlots;    // [2] accumulator complete
   uint64_t* acc_empty = acc_full + 2;         // [2] accumulator drained by both CTAs (leader)
   uint64_t* ovl_free = acc_empty + 2;         // [1] shared columns drained by both (leader)
   uint64_t* mma_done = ovl_free + 1;          // [1] all MMAs of the pair done (leader)
@@ -497,7 +496,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     }
     for (int b = 0; b < kSfSlots; ++b) {
       mbar_init(smem_u32(&sf_full[b]), 2 * kSfWarps);
-      mbar_init(smem_u32(&sf_empty[b]), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&acc_full[b]), 1);
@@ -663,8 +661,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 tc_mma_pair(t_acc, da + 2 * k, db + 2 * k, idesc, t_sf + 4 * k, t_sf + 16 + 8 * k,
                             (kt > 0 || k > 0) ? 1u : 0u);
           }
+          // one commit frees the ring stage and, for the scale warps, the
+          // stage's scale slot (they wait on empty[] two stages back)
           tc_commit_pair(smem_u32(&empty[st]));
-          tc_commit_pair(smem_u32(&sf_empty[slot]));
           if (++st == kStages) {
             st = 0;
             st_ph ^= 1u;
@@ -793,9 +792,15 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       for (int kt = 0; kt < total_kt; ++kt, ++it) {
         const int s = it % kStages;
         const uint32_t slot = it % kSfSlots;
+        // The slot was last used by stage it - 2; its MMAs are done once that
+        // stage's ring barrier completed its phase (the MMA commit and this
+        // warp's own arrival).  That barrier cannot have moved on to its next
+        // phase yet: that needs this warp's arrival for stage it + 3.
+        const uint32_t prev = it - kSfSlots;
         if (!mbar_wait(smem_u32(&sf_in[s]), (it / kStages) & 1u, abort_flag, p.wait_limit_ns) ||
-            !mbar_wait(smem_u32(&sf_empty[slot]), ((it / kSfSlots) & 1u) ^ 1u, abort_flag,
-                       p.wait_limit_ns)) {
+            (it >= (uint32_t)kSfSlots &&
+             !mbar_wait(smem_u32(&empty[prev % kStages]), (prev / kStages) & 1u, abort_flag,
+                        p.wait_limit_ns))) {
           ok = false;
           break;
         }
