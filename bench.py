@@ -47,11 +47,11 @@ QOUT = 0.5 + 1.0 / 16  # bytes written per quantized element (codes + scale byte
 TRAFFIC = {
     # one ncu capture of the full-size step: python bench.py --profile
     # wgrad_step, the first rep's five launches (after the four setup ones)
-    "gemm": {"bytes_per_launch": 867592960 + 156140800,
-             "source_sha256": "8e9e134b290f2562be354aa170c830daca15e84b1f45f6452bf99e03ed875a35"},
-    "encode_x": {"bytes_per_launch": 953817600 + 251720448,
+    "gemm": {"bytes_per_launch": 861515776 + 155492352,
+             "source_sha256": "db997e3f0ca323f1e545cf05e753be64294678a35673c4a110970cdb15f1fdf6"},
+    "encode_x": {"bytes_per_launch": 953861120 + 251800320,
                  "source_sha256": "9934fb8729244c8bf3bcd7f71c02b47b032a710e8124a3f1052c3f65c591eec7"},
-    "amax_x": {"bytes_per_launch": 939637760 + 723968,
+    "amax_x": {"bytes_per_launch": 939543552 + 130304,
                "source_sha256": "9934fb8729244c8bf3bcd7f71c02b47b032a710e8124a3f1052c3f65c591eec7"},
 }
 
