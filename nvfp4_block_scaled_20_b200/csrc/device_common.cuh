@@ -451,19 +451,25 @@ __device__ __forceinline__ void quantize_block16(const float y[16], const ScaleC
 // reciprocal's range) the block takes the exact path.
 constexpr float kPickMargin = 0x1p-10f;
 
-// The E2M1 values of a packed pair of quotients, as fp32x2 (exact): one
-// conversion to the code pair, one back to half precision, two widenings.
-__device__ __forceinline__ uint64_t e2m1_round_pair(uint64_t q) {
+// q - v(q) for a packed pair of quotients, v the E2M1 value: the code pair's
+// half-precision values enter through mixed-precision fused multiply-adds
+// (-1 * v + q, rounded once to fp32), the same fp32 numbers as widening v
+// and subtracting.
+__device__ __forceinline__ uint64_t e2m1_diff_pair(uint64_t q) {
   float lo, hi;
   unpack2(q, lo, hi);
-  uint32_t h2;
+  float dlo, dhi;
   asm("{ .reg .b8 c;\n"
-      "cvt.rn.satfinite.e2m1x2.f32 c, %1, %2;\n"
-      "cvt.rn.f16x2.e2m1x2 %0, c; }"
-      : "=r"(h2)
-      : "f"(hi), "f"(lo));
-  return pack2(__half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu))),
-               __half2float(__ushort_as_half((unsigned short)(h2 >> 16))));
+      ".reg .b32 h2;\n"
+      ".reg .b16 vl, vh;\n"
+      "cvt.rn.satfinite.e2m1x2.f32 c, %3, %2;\n"
+      "cvt.rn.f16x2.e2m1x2 h2, c;\n"
+      "mov.b32 {vl, vh}, h2;\n"
+      "fma.rn.f32.f16 %0, vl, %4, %2;\n"
+      "fma.rn.f32.f16 %1, vh, %4, %3; }"
+      : "=f"(dlo), "=f"(dhi)
+      : "f"(lo), "f"(hi), "h"((unsigned short)0xBC00u));
+  return pack2(dlo, dhi);
 }
 
 // sum_i (q_i - v_i)^2 over 16 elements, q = y * r, v = the E2M1 value of q.
@@ -472,8 +478,7 @@ __device__ __forceinline__ float approx_err16(const float y[16], float r) {
   uint64_t acc[2] = {0ull, 0ull};
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    const uint64_t q = mul2(pack2(y[2 * k], y[2 * k + 1]), rr);
-    const uint64_t d = sub2(q, e2m1_round_pair(q));
+    const uint64_t d = e2m1_diff_pair(mul2(pack2(y[2 * k], y[2 * k + 1]), rr));
     acc[k & 1] = fma2(d, d, acc[k & 1]);
   }
   float a0, a1, b0, b1;
@@ -649,8 +654,7 @@ __device__ __forceinline__ float approx_err16_pairs(const uint64_t yy[8], float 
   uint64_t acc[2] = {0ull, 0ull};
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    const uint64_t q = mul2(yy[k], rr);
-    const uint64_t d = sub2(q, e2m1_round_pair(q));
+    const uint64_t d = e2m1_diff_pair(mul2(yy[k], rr));
     acc[k & 1] = fma2(d, d, acc[k & 1]);
   }
   float a0, a1;
