@@ -661,6 +661,107 @@ __global__ void __launch_bounds__(kThreads, 3)
   pdl_trigger();
 }
 
+// The amax pass of a contiguous tensor (row blocks, no RHT) through shared
+// memory: the tensor's bytes as 16 KB chunks, each one cp.async.bulk into a
+// 4-deep ring per CTA (chunk i of this CTA into slot i % 4), the same bounded
+// waits and drain as the tiled loop.  The last chunk may be shorter (a
+// multiple of 32 bytes).  fn(slot, bytes) reads the chunk.
+template <int kStages, typename F>
+__device__ bool bulk_chunk_loop(const uint8_t* src, uint64_t n_bytes, const Slice sl,
+                                uint8_t* smem, uint32_t* err, F&& fn) {
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kTmaTileBytes);
+  __shared__ int abort_flag;
+  const uint64_t nchunks = (n_bytes + kTmaTileBytes - 1) / kTmaTileBytes;
+  const uint32_t mine =
+      sl.cta < nchunks ? (uint32_t)((nchunks - sl.cta + sl.ncta - 1) / sl.ncta) : 0u;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&full[i])) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    abort_flag = 0;
+  }
+  __syncthreads();
+  auto bytes_of = [&](uint32_t i) {
+    const uint64_t off = (uint64_t)(sl.cta + (uint64_t)i * sl.ncta) * kTmaTileBytes;
+    const uint64_t left = n_bytes - off;
+    return (uint32_t)(left < (uint64_t)kTmaTileBytes ? left : (uint64_t)kTmaTileBytes);
+  };
+  auto issue = [&](uint32_t i) {  // thread 0
+    const uint64_t off = (uint64_t)(sl.cta + (uint64_t)i * sl.ncta) * kTmaTileBytes;
+    const uint32_t bar = smem_addr(&full[i % kStages]), nb = bytes_of(i);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(nb)
+                 : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(smem + (i % kStages) * kTmaTileBytes)),
+        "l"(src + off), "r"(nb), "r"(bar)
+        : "memory");
+  };
+  uint32_t issued = 0;
+  if (threadIdx.x == 0)
+    for (; issued < mine && issued < (uint32_t)kStages - 1; ++issued) issue(issued);
+  bool ok = true;
+  for (uint32_t i = 0; i < mine; ++i) {
+    if (threadIdx.x == 0 && issued < mine) issue(issued++);  // the slot freed by chunk i - 1
+    if (!bar_wait(smem_addr(&full[i % kStages]), (i / kStages) & 1u, kTmaWaitNs)) {
+      abort_flag = 1;
+    } else {
+      fn(smem + (i % kStages) * kTmaTileBytes, bytes_of(i));
+    }
+    __syncthreads();  // every thread is done with slot i before it is refilled
+    if (abort_flag) {
+      ok = false;
+      break;
+    }
+  }
+  if (!ok && threadIdx.x == 0) {
+    atomicOr(err, kDevErrTimeout);
+    for (uint32_t j = issued > (uint32_t)kStages ? issued - kStages : 0u; j < issued; ++j)
+      bar_wait(smem_addr(&full[j % kStages]), (j / kStages) & 1u, kTmaDrainNs);
+  }
+  return ok;
+}
+
+// Thread t reads 16-byte words t, t + 256, ... of a chunk (a warp reads 512
+// contiguous bytes per load: no bank conflicts).
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 3) amax_flat_bulk_kernel(const __grid_constant__ QBatch p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int t = blockIdx.y;
+  const QTensor& q = p.t[t];
+  const Slice sl{blockIdx.x, gridDim.x};
+  const uint64_t n_bytes = (uint64_t)q.rows * (uint64_t)q.cols * sizeof(T);
+  uint32_t m2 = 0u;  // bf16: max |x| per half, as bits
+  float mf = 0.0f;
+  bulk_chunk_loop<kTmaStages>(static_cast<const uint8_t*>(q.x), n_bytes, sl, smem, p.err,
+                              [&](const uint8_t* chunk, uint32_t bytes) {
+    const uint4* c4 = reinterpret_cast<const uint4*>(chunk);
+    const uint32_t nw = bytes >> 4;
+#pragma unroll
+    for (uint32_t k = 0; k < (uint32_t)kTmaTileBytes / 16 / kThreads; ++k) {
+      const uint32_t i = threadIdx.x + k * kThreads;
+      if (i < nw) {
+        const uint4 v = c4[i];
+        if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+          m2 = absmax_bf16x2(m2, v.x);
+          m2 = absmax_bf16x2(m2, v.y);
+          m2 = absmax_bf16x2(m2, v.z);
+          m2 = absmax_bf16x2(m2, v.w);
+        } else {
+          mf = fmaxf(mf, fmaxf(fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))),
+                               fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w)))));
+        }
+      }
+    }
+  });
+  float m = std::is_same<T, __nv_bfloat16>::value
+                ? fmaxf(__uint_as_float(m2 << 16), __uint_as_float(m2 & 0xFFFF0000u))
+                : mf;
+  m = block_reduce_max(m);
+  if (threadIdx.x == 0) p.partials[t * kMaxAmaxCtas + sl.cta] = m;
+  pdl_trigger();
+}
+
 template <bool RHT>
 __global__ void __launch_bounds__(kThreads, NVFP4_COLS_MINB)
     encode_cols_tma_kernel(const __grid_constant__ QBatch p, const __grid_constant__ ColsMaps maps,
@@ -1223,6 +1324,35 @@ cudaError_t launch_ex(K kern, dim3 grid, cudaStream_t s, bool pdl, Args... args)
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// Every tensor of the batch contiguous (ld == cols), 16-byte aligned and with
+// whole 32-byte rows of blocks: the bulk-copy amax pass applies.
+inline bool flat_bulk_ok(const QBatch& b) {
+  for (int i = 0; i < b.n; ++i) {
+    const QTensor& q = b.t[i];
+    if (q.ld != q.cols || ((uintptr_t)q.x & 15u) || q.rows < 1 || q.cols < 1) return false;
+  }
+  return true;
+}
+
+// The bulk-copy amax pass for element type T (its shared-memory attribute is
+// set once per instantiation).
+template <typename T>
+cudaError_t launch_amax_flat(dim3 grid, cudaStream_t s, const QBatch& b) {
+  const int smem_bytes = tma_smem_bytes(kTmaStages);
+  static const bool attr_ok =
+      cudaFuncSetAttribute(amax_flat_bulk_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem_bytes) == cudaSuccess;
+  if (!attr_ok) return cudaErrorNotSupported;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem_bytes;
+  cfg.stream = s;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  return cudaLaunchKernelEx(&cfg, amax_flat_bulk_kernel<T>, b);
+}
+
 template <typename T, int MODE, bool RHT>
 cudaError_t launch_mode(const QBatch& b, cudaStream_t s) {
   const uint64_t units = max_units(b, MODE);
@@ -1237,7 +1367,23 @@ cudaError_t launch_mode(const QBatch& b, cudaStream_t s) {
     uint64_t cap = (uint64_t)num_sms() * 3;
     if (cap > (uint64_t)kMaxAmaxCtas) cap = kMaxAmaxCtas;
     ga = (int)(want < 1 ? 1 : (want < cap ? want : cap));
-    cudaError_t e = launch_ex(amax_kernel<T, MODE, RHT>, dim3(ga, b.n), s, false, b);
+    cudaError_t e;
+    if (MODE == kModeRows && !RHT && flat_bulk_ok(b)) {
+      // contiguous tensors: 16 KB chunks staged by bulk copies
+      uint64_t chunks = 0;
+      for (int i = 0; i < b.n; ++i) {
+        const uint64_t c = ((uint64_t)b.t[i].rows * (uint64_t)b.t[i].cols * sizeof(T) +
+                            kTmaTileBytes - 1) / kTmaTileBytes;
+        chunks = c > chunks ? c : chunks;
+      }
+      uint64_t cap_b = (uint64_t)num_sms() * 3 / (uint64_t)b.n;
+      if (cap_b > (uint64_t)kMaxAmaxCtas) cap_b = kMaxAmaxCtas;
+      if (cap_b < 1) cap_b = 1;
+      ga = (int)(chunks < cap_b ? (chunks < 1 ? 1 : chunks) : cap_b);
+      e = launch_amax_flat<T>(dim3(ga, b.n), s, b);
+    } else {
+      e = launch_ex(amax_kernel<T, MODE, RHT>, dim3(ga, b.n), s, false, b);
+    }
     if (e != cudaSuccess) return e;
     if (b.amax_only) return launch_ex(finalize_kernel, dim3(b.n), s, true, b, ga);
   }
