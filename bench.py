@@ -47,12 +47,12 @@ QOUT = 0.5 + 1.0 / 16  # bytes written per quantized element (codes + scale byte
 TRAFFIC = {
     # one ncu capture of the full-size step: python bench.py --profile
     # wgrad_step, the first rep's five launches (after the four setup ones)
-    "gemm": {"bytes_per_launch": 861515776 + 155492352,
-             "source_sha256": "db997e3f0ca323f1e545cf05e753be64294678a35673c4a110970cdb15f1fdf6"},
-    "encode_x": {"bytes_per_launch": 953861120 + 251800320,
-                 "source_sha256": "9934fb8729244c8bf3bcd7f71c02b47b032a710e8124a3f1052c3f65c591eec7"},
-    "amax_x": {"bytes_per_launch": 939543552 + 130304,
-               "source_sha256": "9934fb8729244c8bf3bcd7f71c02b47b032a710e8124a3f1052c3f65c591eec7"},
+    "gemm": {"bytes_per_launch": 862240768 + 155704320,
+             "source_sha256": "d29567387e7e5a4f9d75d21ed65204df5f1cb7ee18804480b92e8ea671e1b6e7"},
+    "encode_x": {"bytes_per_launch": 954204160 + 251442176,
+                 "source_sha256": "d443ba1bae7321cd2d15be6d2775c8c68c4ae04fb60685defd54ee1f4596e1ec"},
+    "amax_x": {"bytes_per_launch": 939580928 + 470272,
+               "source_sha256": "d443ba1bae7321cd2d15be6d2775c8c68c4ae04fb60685defd54ee1f4596e1ec"},
 }
 
 
@@ -562,6 +562,8 @@ def main():
         "quantize_x": gbs((4 + QOUT) * n_x, part["quant_x"]),
         "amax_only_x": gbs(2 * n_x, part["amax_x"]),
         "encode_only_x": gbs((2 + QOUT) * n_x, part["encode_x"]),
+        "traffic_bytes": {"gemm": kernel_traffic("gemm"), "encode_x": kernel_traffic("encode_x"),
+                          "amax_x": kernel_traffic("amax_x")},
         "note": "quantize_* = the step's two launches (amax pass, then the encode pass that "
                 "reduces the amax partials into the global scale) counted at the algorithmic "
                 "two-read bytes (4 + 0.5625 B/element); encode_only_* = the encode pass alone "
@@ -584,8 +586,8 @@ def main():
         ach = nb / (part[top] * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
                 "frac": round(ach / hbm, 4), "traffic": kernel_traffic(top),
-                "kernel": ("encode_kernel<bf16, cols, rht> (transposing RHT16 encode of X)"
-                           if top == "encode_x" else "amax_kernel<bf16, cols, rht> of X"),
+                "kernel": ("encode_cols_tma_kernel<rht> (transposing RHT16 encode of X)"
+                           if top == "encode_x" else "amax_cols_tma_kernel<rht> of X"),
                 "peak_source": "%s HBM copy bandwidth" % pk["source"]}
     roof["algorithmic"] = ("GEMM: 2*M*N*K FLOP per launch; encode: 2 B read + 0.5625 B "
                            "written per element; amax: 2 B read per element")
