@@ -37,7 +37,9 @@ WORKLOAD = ("DiT weight gradient of the FFN up projection, W4A4: dY bf16 [32768x
             "(4-vs-6 on) of both; dW = dY^T X [3072x14336] fp32")
 FLUSH_BYTES = 256 << 20
 # our kernels per step: amax + encode for dY, amax + encode for X, the GEMM
-LAUNCHES_PER_STEP = 5
+# library launches per headline step: amax and encode for dY and X, the GEMM,
+# and the GEMM's split-tail reduction when its workspace enables the split
+LAUNCHES_PER_STEP_UNSPLIT = 5
 QOUT = 0.5 + 1.0 / 16  # bytes written per quantized element (codes + scale bytes)
 
 
@@ -46,9 +48,11 @@ QOUT = 0.5 + 1.0 / 16  # bytes written per quantized element (codes + scale byte
 # taken on (hash of the kernel's source files).
 TRAFFIC = {
     # one ncu capture of the full-size step: python bench.py --profile
-    # wgrad_step, the first rep's five launches (after the four setup ones)
-    "gemm": {"bytes_per_launch": 862240768 + 155704320,
-             "source_sha256": "d29567387e7e5a4f9d75d21ed65204df5f1cb7ee18804480b92e8ea671e1b6e7"},
+    # wgrad_step, the first rep's six launches (after the four setup ones);
+    # "gemm" is the GEMM with its split last round plus the reduction of the
+    # split tiles' partial sums (gemm_kernel<true> + split_reduce_kernel)
+    "gemm": {"bytes_per_launch": 889843200 + 158941696 + 18881536 + 0,
+             "source_sha256": "d726cc240ca8c9a4404f585d01cabf1b1364170138dbb3a8f3c1e10376b6a5de"},
     "encode_x": {"bytes_per_launch": 954204160 + 251442176,
                  "source_sha256": "d443ba1bae7321cd2d15be6d2775c8c68c4ae04fb60685defd54ee1f4596e1ec"},
     "amax_x": {"bytes_per_launch": 939580928 + 470272,
@@ -77,6 +81,14 @@ def kernel_traffic(kernel):
     if not rec or rec["source_sha256"] != _sources_digest(KERNEL_SOURCES[kernel]):
         return None
     return rec["bytes_per_launch"]
+
+
+def launches_per_step(nv, ws_g):
+    """Library launches of one headline step: the GEMM adds its split-tail
+    reduction kernel when ws_g is large enough for the split."""
+    from nvfp4_block_scaled_20_b200 import capi
+    split = ws_g.numel() > capi.nvfp4_workspace_bytes(0)
+    return LAUNCHES_PER_STEP_UNSPLIT + (1 if split else 0)
 
 
 def peaks():
@@ -338,16 +350,18 @@ def run_profile_case(name, reps=3):
     dev = torch.device("cuda", 0)
     ws = nv.workspace(8, dev)
 
+    ws_g = ws
     if name == "wgrad_step":
         dy, xw, mask = synth.wgrad(dev)
         qdy = nv.quantize_1d(dy, rht=True, mask=mask, block_axis=1, ws=ws)
         qxw = nv.quantize_1d(xw, rht=True, mask=mask, block_axis=1, ws=ws)
         dw = torch.empty((dy.shape[1], xw.shape[1]), dtype=torch.float32, device=dev)
+        ws_g = nv.gemm_workspace(dy.shape[1], xw.shape[1], dy.shape[0], device=dev)
 
         def run():
             nv.quantize_1d(dy, rht=True, mask=mask, block_axis=1, out=qdy, ws=ws)
             nv.quantize_1d(xw, rht=True, mask=mask, block_axis=1, out=qxw, ws=ws)
-            nv.gemm(qdy, qxw, out=dw, ws=ws)
+            nv.gemm(qdy, qxw, out=dw, ws=ws_g)
     elif name == "qkv_step":
         x, w = synth.qkv_linear(dev)
 
@@ -396,14 +410,15 @@ def run_profile_case(name, reps=3):
         dy, xw, mask = synth.wgrad(dev, t=8192)
         qdy = nv.quantize_1d(dy, rht=True, mask=mask, block_axis=1, ws=ws)
         qxw = nv.quantize_1d(xw, rht=True, mask=mask, block_axis=1, ws=ws)
+        ws_g = nv.gemm_workspace(dy.shape[1], xw.shape[1], dy.shape[0], device=dev)
 
         def run():
-            nv.gemm(qdy, qxw, out_dtype=torch.float32, ws=ws)
+            nv.gemm(qdy, qxw, out_dtype=torch.float32, ws=ws_g)
 
     for _ in range(reps):
         run()
     torch.cuda.synchronize()
-    assert nv.device_error(ws) == 0
+    assert nv.device_error(ws) == 0 and nv.device_error(ws_g) == 0
     print("profile case %s: %s, %d reps" % (name, PROFILE_CASES[name], reps))
     return 0
 
@@ -456,7 +471,9 @@ def main():
     qdy = nv.QTensor(*nv._alloc_q(D_OUT, T_TOK, T, dev), D_OUT, T_TOK, T)
     qxw = nv.QTensor(*nv._alloc_q(D_IN, T_TOK, T, dev), D_IN, T_TOK, T)
     dw = torch.empty((D_OUT, D_IN), dtype=torch.float32, device=dev)
-    ws_dy, ws_x, ws_g = nv.workspace(1, dev), nv.workspace(1, dev), nv.workspace(0, dev)
+    ws_dy, ws_x = nv.workspace(1, dev), nv.workspace(1, dev)
+    # the GEMM's workspace with room for its split last round
+    ws_g = nv.gemm_workspace(D_OUT, D_IN, T_TOK, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     flush_rd = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_sink = torch.empty((), dtype=torch.float32, device=dev)
@@ -578,7 +595,9 @@ def main():
         roof = {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp4_peak, 1),
                 "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_peak, 4),
                 "traffic": kernel_traffic("gemm"),
-                "kernel": "gemm_kernel (CTA-pair tcgen05.mma kind::mxf4nvf4), 3072x14336x32768",
+                "kernel": ("gemm_kernel (CTA-pair tcgen05.mma kind::mxf4nvf4), 3072x14336x32768"
+                           + (", last round split along K + split_reduce_kernel"
+                              if launches_per_step(nv, ws_g) > LAUNCHES_PER_STEP_UNSPLIT else "")),
                 "peak_source": "%s bf16 burst %.1f TFLOP/s x 4 (nominal dense FP4:BF16 "
                                "ratio)" % (pk["source"], pk["bf16_tflops"])}
     else:
@@ -635,7 +654,7 @@ def main():
                        "timing": "CUDA events around a CUDA-graph replay of the step, max over ranks"},
             "roofline": roof,
             "breakdown": breakdown,
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "gpu_launches": launches_per_step(nv, ws_g) * args.steps,
             "clocks": clk,
         }
         if rows:
@@ -735,7 +754,8 @@ def measure_rows(nv, synth, torch, dev, stream, timed, pk, reps):
     nv.quantize_1d(h, out=qh, ws=ws, stream=stream)
     g_up = tc(lambda: nv.gemm(qx, qu, out=h, epilogue=nv.NVFP4_EPI_GELU_TANH, ws=ws,
                               stream=stream), 2.0 * Mf * Hd * D)
-    g_dn = tc(lambda: nv.gemm(qh, qd, out=y, ws=ws, stream=stream), 2.0 * Mf * D * Hd)
+    ws_dn = nv.gemm_workspace(Mf, D, Hd, device=dev)  # the down GEMM splits its last round
+    g_dn = tc(lambda: nv.gemm(qh, qd, out=y, ws=ws_dn, stream=stream), 2.0 * Mf * D * Hd)
 
     ws_h = nv.workspace(1, dev)
 
@@ -744,7 +764,7 @@ def measure_rows(nv, synth, torch, dev, stream, timed, pk, reps):
         # the up GEMM leaves H's amax in ws_h: H's quantization is one encode pass
         nv.gemm(qx, qu, out=h, epilogue=nv.NVFP4_EPI_GELU_TANH, amax_ws=ws_h, stream=stream)
         nv.quantize_1d(h, out=qh, ws=ws_h, amax_ready=True, stream=stream)
-        nv.gemm(qh, qd, out=y, ws=ws, stream=stream)
+        nv.gemm(qh, qd, out=y, ws=ws_dn, stream=stream)
 
     ffn = tc(ffn_step, 4.0 * Mf * Hd * D)
     ffn["note"] = ("quantize X, up GEMM + GELU recording H's amax, encode H (no amax pass), "
@@ -860,7 +880,7 @@ def measure_rows(nv, synth, torch, dev, stream, timed, pk, reps):
         "60 tensors, 24 heads x (3 + 3 + 9 of 21 frames), one launch")
     del kv, kq, kout
     assert (nv.device_error(ws, stream) == 0 and nv.device_error(ws_h, stream) == 0
-            and nv.device_error(ws_kv, stream) == 0)
+            and nv.device_error(ws_kv, stream) == 0 and nv.device_error(ws_dn, stream) == 0)
     torch.cuda.empty_cache()
     return out
 

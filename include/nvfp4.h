@@ -330,13 +330,27 @@ NVFP4_API nvfp4_status nvfp4_dequantize_rows(const nvfp4_tensor_desc* descs, int
  *            qp->amax_from_workspace = 1 skips its amax pass and gives the
  *            same codes, scales and global scale as without it.
  * Shape: M >= 1, N % 16 == 0, K % 64 == 0, ldo >= N, ldo * elem % 16 == 0.
- * Workspace: nvfp4_workspace_bytes(0) (the device error word). */
+ * Workspace: nvfp4_workspace_bytes(0) (the device error word) at least.
+ * With nvfp4_gemm_workspace_bytes(M, N, K, epilogue) bytes, 16-byte aligned,
+ * the tiles of the persistent schedule's last, partial round are each split
+ * along K among otherwise idle SM pairs (long K, plain epilogue only): their
+ * fp32 partial sums go to the workspace and a second kernel on the same
+ * stream adds them in a fixed order, scales and stores them.  The result is
+ * deterministic; against the unsplit kernel it differs only by the order of
+ * the fp32 additions over K. */
 NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf,
                         const float* a_alpha, const uint8_t* b_codes,
                         const uint8_t* b_sf, const float* b_alpha, int64_t M,
                         int64_t N, int64_t K, void* out, int32_t out_dtype,
                         int64_t ldo, int32_t epilogue, void* workspace,
                         size_t workspace_bytes, void* stream);
+
+/* Workspace bytes with which nvfp4_gemm splits its last partial round for
+ * this shape and epilogue (room for the error word, the amax partials and
+ * one fp32 256 x 256 slab per split unit); nvfp4_workspace_bytes of the call
+ * when the launch would not split.  Depends on the current device's SM
+ * count; without a usable device, nvfp4_workspace_bytes of the call. */
+NVFP4_API size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t epilogue);
 
 /* Bytes of the scratch nvfp4_gemm_lora needs for an M-row activation and a
  * rank-`rank` adapter (the scaled adapter input, bf16 [M, 2 rank]). */

@@ -63,6 +63,17 @@ def workspace(n_tensors: int = 1, device=None):
                        device=device or "cuda")
 
 
+def gemm_workspace(M: int, N: int, K: int, epilogue: int = NVFP4_EPI_NONE, device=None):
+    """Workspace for gemm(): nvfp4_gemm_workspace_bytes, error word zeroed (the
+    rest needs no initialization).  With it, the tiles of the last partial
+    round of the persistent schedule are split along K."""
+    torch = _torch()
+    ws = torch.empty(capi.nvfp4_gemm_workspace_bytes(M, N, K, epilogue), dtype=torch.uint8,
+                     device=device or "cuda")
+    ws[:capi.nvfp4_workspace_bytes(0)].zero_()
+    return ws
+
+
 def _qparams(four_over_six, rht, mask, block_axis, sf_layout, alpha_in, amax_ready=False):
     return capi.nvfp4_qparams(int(four_over_six), int(rht), int(mask) & 0xFFFFFFFF,
                               int(block_axis), int(sf_layout), int(bool(amax_ready)),
@@ -256,7 +267,7 @@ def gemm(a: QTensor, b: QTensor, out_dtype=None, epilogue=NVFP4_EPI_NONE, out=No
         if ws is not None and ws is not amax_ws:
             raise ValueError("with amax_ws the GEMM uses that workspace")
         ws, epilogue = amax_ws, epilogue | NVFP4_EPI_AMAX
-    ws = workspace(0, a.codes.device) if ws is None else ws
+    ws = gemm_workspace(M, N, K, epilogue, a.codes.device) if ws is None else ws
     code = NVFP4_BF16 if out.dtype == torch.bfloat16 else NVFP4_F32
     st = capi.nvfp4_gemm(a.codes.data_ptr(), a.scales.data_ptr(), a.alpha.data_ptr(),
                          b.codes.data_ptr(), b.scales.data_ptr(), b.alpha.data_ptr(), M, N, K,

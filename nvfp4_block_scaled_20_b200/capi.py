@@ -26,7 +26,7 @@ EXPORTED = [
     "nvfp4_transpose_2d",
     "nvfp4_gemm", "nvfp4_rht16", "nvfp4_get_device_error", "nvfp4_status_string",
     "nvfp4_convert_sweep", "nvfp4_set_wait_limit", "nvfp4_set_test_stall",
-    "nvfp4_lora_scratch_bytes", "nvfp4_gemm_lora",
+    "nvfp4_lora_scratch_bytes", "nvfp4_gemm_lora", "nvfp4_gemm_workspace_bytes",
 ]
 
 
@@ -79,6 +79,7 @@ _SIGS = {
     "nvfp4_set_wait_limit": (_I32, [ctypes.c_uint64]),
     "nvfp4_set_test_stall": (_I32, [_I32]),
     "nvfp4_lora_scratch_bytes": (_SZ, [_I64, _I64]),
+    "nvfp4_gemm_workspace_bytes": (_SZ, [_I64, _I64, _I64, _I32]),
     "nvfp4_gemm_lora": (_I32, [_V, _V, _V, _V, _V, _V, _I64, _I64, _I64, _V, _I64, _V, _I64, _I64,
                                ctypes.c_float, _V, _SZ, _V, _I32, _I64, _I32, _V, _SZ, _V]),
 }
@@ -170,6 +171,10 @@ def nvfp4_gemm(a_codes, a_sf, a_alpha, b_codes, b_sf, b_alpha, M, N, K, out, out
                epilogue, ws, ws_bytes, stream):
     return _call("nvfp4_gemm", a_codes, a_sf, a_alpha, b_codes, b_sf, b_alpha, M, N, K, out,
                  out_dtype, ldo, epilogue, ws, ws_bytes, stream)
+
+
+def nvfp4_gemm_workspace_bytes(M, N, K, epilogue):
+    return _call("nvfp4_gemm_workspace_bytes", M, N, K, epilogue)
 
 
 def nvfp4_lora_scratch_bytes(M, rank):

@@ -23,6 +23,11 @@ inline cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
 // Workspace layout: [0, 4) device error word, then kMaxAmaxCtas fp32
 // partial maxima per tensor from 256 on.  Nothing in it needs clearing.
 uint32_t* err_word(void* ws) { return static_cast<uint32_t*>(ws); }
+// nvfp4_gemm's partial-sum slabs (the split last round) follow the error word
+// and one tensor's amax partials, 1 KB aligned; one slab is an fp32 256 x 256
+// tile.
+constexpr size_t kSlabOffset = (kErrWordBytes + kMaxAmaxCtas * sizeof(float) + 1023) / 1024 * 1024;
+constexpr size_t kSlabBytes = 256 * 256 * sizeof(float);
 float* partials(void* ws) {
   return reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kErrWordBytes);
 }
@@ -344,6 +349,12 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
                      epilogue, ws, ws_bytes, stream, nullptr);
 }
 
+size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t epilogue) {
+  const size_t base = nvfp4_workspace_bytes((epilogue & NVFP4_EPI_AMAX) ? 1 : 0);
+  const int64_t slabs = gemm_split_slabs(M, N, K, epilogue);
+  return slabs > 0 ? kSlabOffset + (size_t)slabs * kSlabBytes : base;
+}
+
 size_t nvfp4_lora_scratch_bytes(int64_t M, int64_t rank) {
   return (M > 0 && rank > 0) ? (size_t)M * (size_t)rank * 4u : 0u;
 }
@@ -417,6 +428,12 @@ nvfp4_status gemm_common(const uint8_t* a_codes, const uint8_t* a_sf, const floa
   g.lora_b = nullptr;
   g.rank = 0;
   g.u_scaled = nullptr;
+  g.slabs = nullptr;
+  g.slab_cap = 0;
+  if (!lora && ws_bytes >= kSlabOffset + kSlabBytes && aligned(ws, 16)) {
+    g.slabs = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kSlabOffset);
+    g.slab_cap = (int64_t)((ws_bytes - kSlabOffset) / kSlabBytes);
+  }
   if (lora) {
     g.lora_u = lora->lora_u;
     g.lora_b = lora->lora_b;

@@ -214,6 +214,13 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
       "r"(src), "r"(c0), "r"(c1)
       : "memory");
 }
+// Untiled copy of `bytes` (a multiple of 16, both addresses 16-byte
+// aligned) from this CTA's shared memory to global memory, in the bulk group.
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src),
+               "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -390,6 +397,15 @@ struct Params {
   // each a 128-byte column chunk (64 bf16) of the scaled adapter input U'
   // [M, 2r] (hi and lo halves) and of B_lora [N, r] (chunk c mod lora_kt / 2)
   int32_t lora_kt;
+  // Work units: [0, full_tiles) are whole tiles; each of the next tail_tiles
+  // tiles is cut into split_s ranges of K stages, one unit per range, whose
+  // fp32 partial sums go to slab (unit - full_tiles) of `slabs` for
+  // split_reduce_kernel.  No split: full_tiles = all tiles, tail_tiles = 0,
+  // split_s = 1.  A slab is 256 x 256 fp32 in 2 KB blocks of 32 rows x 16
+  // columns (row-major inside), block (row / 32, column / 16) at
+  // ((row / 32) * 16 + column / 16) * 2 KB: one epilogue staging chunk each.
+  int32_t full_tiles, tail_tiles, split_s;
+  float* slabs;
 };
 
 // Tile t of the grouped raster -> (tile row, tile column).
@@ -401,6 +417,29 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mt
   const int r = t - g * per_group;
   mt = first_m + r % gm;
   nt = r / gm;
+}
+
+// Work unit u: its tile, its K stages [kt0, kt1) and its partial-sum slab
+// (-1: a whole tile, stored to the output).
+struct Unit {
+  int tile, kt0, kt1, slab;
+};
+template <bool kSplit>
+__device__ __forceinline__ Unit unit_of(const Params& p, int u, int num_kt, int total_kt) {
+  Unit w;
+  if (!kSplit || u < p.full_tiles) {
+    w.tile = u;
+    w.kt0 = 0;
+    w.kt1 = total_kt;
+    w.slab = -1;
+  } else {
+    const int v = u - p.full_tiles, i = v / p.split_s, j = v - i * p.split_s;
+    w.tile = p.full_tiles + i;
+    w.kt0 = j * num_kt / p.split_s;
+    w.kt1 = (j + 1) * num_kt / p.split_s;
+    w.slab = v;
+  }
+  return w;
 }
 
 // max(|a|, |b|) per bf16 half of two packed words (sign bits cleared).
@@ -450,6 +489,16 @@ __device__ __forceinline__ void stage16(const Params& p, uint8_t* chunk, int lan
   }
 }
 
+// A split unit's lane: its 16 unscaled fp32 sums as its row of the chunk.
+__device__ __forceinline__ void stage16_raw(uint8_t* chunk, int lane, const uint32_t r[16]) {
+  uint4* d4 = reinterpret_cast<uint4*>(chunk + lane * 64);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d4[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+}
+
+// kSplit: the launch has split units (a separate instance, so that the
+// common unsplit launch carries none of their code).
+template <bool kSplit>
 __global__ void __launch_bounds__(kNumThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmU,
@@ -482,9 +531,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
   const int num_m = (p.M + 2 * BM - 1) / (2 * BM), num_n = (p.N + BN - 1) / BN;
-  const int num_tiles = num_m * num_n;
   const int num_kt = (p.K + BK - 1) / BK;
   const int total_kt = num_kt + p.lora_kt;  // FP4 stages, then the LoRA stages of a tile
+  const int num_units = kSplit ? p.full_tiles + p.tail_tiles * p.split_s : num_m * num_n;
   const int kgroups = p.K / 64;  // 4-block scale groups per 128-row band
   const int mbands_total = (p.M + 127) / 128, nbands_total = (p.N + 127) / 128;
 
@@ -531,12 +580,13 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     if (lane == 0) {
       uint32_t it = 0;
       bool ok = true;
-      for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+      for (int u = pair; u < num_units && ok; u += num_pairs) {
+        const Unit w = unit_of<kSplit>(p, u, num_kt, total_kt);
         int mt, nt;
-        tile_coords(t, num_m, num_n, mt, nt);
+        tile_coords(w.tile, num_m, num_n, mt, nt);
         const int m0 = mt * 2 * BM + (int)rank * BM, nb0 = nt * BN + (int)rank * (BN / 2);
         const int mband = mt * 2 + (int)rank;
-        for (int kt = 0; kt < total_kt; ++kt, ++it) {
+        for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
           const int s = it % kStages;
           const uint32_t round = it / kStages;
           if (!mbar_wait(smem_u32(&empty[s]), (round & 1u) ^ 1u, abort_flag, p.wait_limit_ns)) {
@@ -619,7 +669,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       // test hook (nvfp4_set_test_stall): a wait that runs out after the
       // pipeline bound while the producers' first stages are in flight
       if (p.stall && !mbar_wait(smem_u32(never), 0, abort_flag, p.wait_limit_ns)) ok = false;
-      for (int t = pair; t < num_tiles && ok; t += num_pairs, ++tile_i) {
+      for (int u = pair; u < num_units && ok; u += num_pairs, ++tile_i) {
+        const Unit w = unit_of<kSplit>(p, u, num_kt, total_kt);
         const uint32_t b = tile_i & 1u, use = tile_i >> 1;
         // accumulator b drained by both CTAs' epilogues of tile_i - 2, and
         // the shared columns by those of tile_i - 1
@@ -633,7 +684,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         }
         tc_fence_after();
         const uint32_t t_acc = tmem + (b ? kAcc1Col : 0u);
-        for (int kt = 0; kt < total_kt; ++kt, ++it) {
+        for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
           if (!mbar_wait(smem_u32(&full[st]), st_ph, abort_flag, p.wait_limit_ns) ||
               !mbar_wait(smem_u32(&sf_full[slot]), slot_ph, abort_flag, p.wait_limit_ns)) {
             ok = false;
@@ -659,7 +710,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             for (int k = 0; k < 4; ++k)
               if (k < nmma)
                 tc_mma_pair(t_acc, da + 2 * k, db + 2 * k, idesc, t_sf + 4 * k, t_sf + 16 + 8 * k,
-                            (kt > 0 || k > 0) ? 1u : 0u);
+                            (kt > w.kt0 || k > 0) ? 1u : 0u);
           }
           // one commit frees the ring stage and, for the scale warps, the
           // stage's scale slot (they wait on empty[] two stages back)
@@ -692,10 +743,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     uint32_t tile_i = 0, chunk_i = 0;
     const bool want_amax = p.amax_partials != nullptr;
     uint32_t lane_amax = 0u;  // bf16x2 pair (bf16 out) or fp32 bits (fp32 out), both >= 0
-    for (int t = pair; t < num_tiles; t += num_pairs, ++tile_i) {
+    for (int u = pair; u < num_units; u += num_pairs, ++tile_i) {
+      const Unit w = unit_of<kSplit>(p, u, num_kt, total_kt);
       const uint32_t b = tile_i & 1u, use = tile_i >> 1;
       int mt, nt;
-      tile_coords(t, num_m, num_n, mt, nt);
+      tile_coords(w.tile, num_m, num_n, mt, nt);
       const int m0 = mt * 2 * BM + (int)rank * BM, n0 = nt * BN;
       if (!mbar_wait(smem_u32(&acc_full[b]), use & 1u, abort_flag, p.wait_limit_ns)) {
         atomicOr(p.err, kDevErrTimeout);
@@ -720,11 +772,18 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         uint8_t* chunk = my_stage + (chunk_i & 1u) * kEpiChunkBytes;
         if (lane == 0) bulk_wait_read_one();  // this buffer's previous store has read it
         __syncwarp();
-        stage16(p, chunk, lane, r, scale, want_amax && m0 + quad * 32 + lane < p.M, lane_amax);
+        if (!kSplit || w.slab < 0)
+          stage16(p, chunk, lane, r, scale, want_amax && m0 + quad * 32 + lane < p.M, lane_amax);
+        else
+          stage16_raw(chunk, lane, r);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmOut, smem_u32(chunk), n0 + c, m0 + quad * 32);
+          if (!kSplit || w.slab < 0)
+            tma_store_2d(&tmOut, smem_u32(chunk), n0 + c, m0 + quad * 32);
+          else  // the chunk is one 2 KB block of the unit's slab
+            bulk_store(p.slabs + ((size_t)(w.slab * 8 + (int)rank * 4 + quad) * 16 + c / 16) * 512,
+                       smem_u32(chunk), kEpiChunkBytes);
           bulk_commit();
         }
         ++chunk_i;
@@ -788,8 +847,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     uint32_t it = 0;
     bool ok = true;
-    for (int t = pair; t < num_tiles && ok; t += num_pairs) {
-      for (int kt = 0; kt < total_kt; ++kt, ++it) {
+    for (int u = pair; u < num_units && ok; u += num_pairs) {
+      const Unit w = unit_of<kSplit>(p, u, num_kt, total_kt);
+      for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
         const int s = it % kStages;
         const uint32_t slot = it % kSfSlots;
         // The slot was last used by stage it - 2; its MMAs are done once that
@@ -932,6 +992,49 @@ bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_
   return r == CUDA_SUCCESS;
 }
 
+// The split tiles: out = a_alpha b_alpha * (slab 0 + slab 1 + ... + slab S-1)
+// of each, summed in slab order (fp32), then rounded to the output type as
+// the GEMM's epilogue does; rows past M and columns past N are not stored.
+// kReduceRows rows of a 256-column tile per block, four columns per thread.
+constexpr int kReduceRows = 4;
+__global__ void __launch_bounds__(kReduceRows * (BN / 4))
+    split_reduce_kernel(const float* __restrict__ slabs, const Params p, int num_m, int num_n) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  constexpr int kBlocksPerTile = 2 * BM / kReduceRows;
+  const int i = blockIdx.x / kBlocksPerTile;
+  const int r = (blockIdx.x % kBlocksPerTile) * kReduceRows + threadIdx.x / (BN / 4);
+  const int c = (threadIdx.x % (BN / 4)) * 4;
+  int mt, nt;
+  tile_coords(p.full_tiles + i, num_m, num_n, mt, nt);
+  const int m = mt * 2 * BM + r, n = nt * BN + c;
+  if (m >= p.M || n >= p.N) return;  // N % 16 == 0: columns n .. n + 3 all inside
+  // slab block (r / 32, c / 16), row r % 32, columns c % 16 .. + 3
+  const float4* src = reinterpret_cast<const float4*>(
+      slabs + (size_t)i * p.split_s * 2 * BM * BN + ((r / 32) * 16 + c / 16) * 512 + (r % 32) * 16 +
+      c % 16);
+  constexpr size_t kSlabF4 = (size_t)2 * BM * BN / 4;
+  float4 acc = src[0];
+  for (int j = 1; j < p.split_s; ++j) {
+    const float4 v = src[j * kSlabF4];
+    acc.x = __fadd_rn(acc.x, v.x);
+    acc.y = __fadd_rn(acc.y, v.y);
+    acc.z = __fadd_rn(acc.z, v.z);
+    acc.w = __fadd_rn(acc.w, v.w);
+  }
+  const float scale = __fmul_rn(*p.a_alpha, *p.b_alpha);
+  const float4 o = make_float4(__fmul_rn(acc.x, scale), __fmul_rn(acc.y, scale),
+                               __fmul_rn(acc.z, scale), __fmul_rn(acc.w, scale));
+  if (p.out_bf16) {
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(o.x, o.y), h1 = __floats2bfloat162_rn(o.z, o.w);
+    uint2 w;
+    w.x = *reinterpret_cast<uint32_t*>(&h0);
+    w.y = *reinterpret_cast<uint32_t*>(&h1);
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + (size_t)m * p.ldo + n) = w;
+  } else {
+    *reinterpret_cast<float4*>(static_cast<float*>(p.out) + (size_t)m * p.ldo + n) = o;
+  }
+}
+
 cudaLaunchConfig_t pair_config(dim3 grid, cudaStream_t s, cudaLaunchAttribute attr[2]) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -964,6 +1067,56 @@ bool make_out_map(CUtensorMap* map, void* out, int64_t M, int64_t N, int64_t ldo
                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Resident pairs: one pair per two SMs where the GPU's layout allows.
+int max_resident_pairs() {
+  static const int n_pairs = [] {
+    if (cudaFuncSetAttribute(gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes) != cudaSuccess)
+      return 0;
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = pair_config(dim3(2), nullptr, attr);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel<false>, &cfg) != cudaSuccess || n < 1)
+      n = num_sms() / 2;
+    return n;
+  }();
+  return n_pairs;
+}
+
+// Split of the last, partial round of the persistent schedule: with `tiles`
+// tiles on P resident pairs, the first tiles - tiles % P run whole; each of
+// the rest is cut into S K ranges (S <= P / (tiles % P), at least
+// kSplitMinStages stages each) run by otherwise idle pairs, so the launch
+// ends after about tiles / P tile times instead of ceil(tiles / P).  Only
+// for long K (a tile time worth more than the extra reduction launch), plain
+// epilogues and no LoRA branch; at most slab_cap partial tiles.
+constexpr int kSplitMinKt = 32;      // K >= 8192
+constexpr int kSplitMinStages = 8;   // K stages per split unit
+struct SplitPlan {
+  int full_tiles, tail_tiles, split_s, pairs;
+};
+SplitPlan plan_split(int64_t M, int64_t N, int64_t K, bool eligible, int64_t slab_cap) {
+  const int64_t tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + BN - 1) / BN);
+  const int64_t num_kt = (K + BK - 1) / BK;
+  const int P = max_resident_pairs();
+  SplitPlan sp{(int)tiles, 0, 1, (int)(tiles < P ? tiles : P)};
+  if (!eligible || P < 2 || num_kt < kSplitMinKt) return sp;
+  const int64_t rem = tiles % P;
+  if (rem == 0) return sp;
+  int64_t S = P / rem;
+  if (S > num_kt / kSplitMinStages) S = num_kt / kSplitMinStages;
+  if (S * rem > slab_cap) S = slab_cap / rem;
+  if (S < 2) return sp;
+  sp.full_tiles = (int)(tiles - rem);
+  sp.tail_tiles = (int)rem;
+  sp.split_s = (int)S;
+  const int64_t units = sp.full_tiles + rem * S;
+  sp.pairs = (int)(units < P ? units : P);
+  return sp;
 }
 
 int launch_persistent(const GemmArgs& a, cudaStream_t s) {
@@ -1008,24 +1161,31 @@ int launch_persistent(const GemmArgs& a, cudaStream_t s) {
   p.wait_limit_ns = a.wait_limit_ns;
   p.stall = a.stall;
   p.lora_kt = lora_kt;
-  // resident pairs: one pair per two SMs where the GPU's layout allows
-  static const int max_pairs = [] {
-    if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes) != cudaSuccess)
-      return 0;
-    cudaLaunchAttribute attr[2];
-    cudaLaunchConfig_t cfg = pair_config(dim3(2), nullptr, attr);
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel, &cfg) != cudaSuccess || n < 1)
-      n = num_sms() / 2;
-    return n;
-  }();
-  if (max_pairs < 1) return (int)cudaErrorInvalidConfiguration;
-  const int64_t tiles = ((a.M + 2 * BM - 1) / (2 * BM)) * ((a.N + BN - 1) / BN);
-  const int pairs = (int)(tiles < max_pairs ? tiles : max_pairs);
+  if (max_resident_pairs() < 1) return (int)cudaErrorInvalidConfiguration;
+  const SplitPlan sp = plan_split(a.M, a.N, a.K, lora_kt == 0 && a.epilogue == 0 && a.slabs,
+                                  a.slab_cap);
+  p.full_tiles = sp.full_tiles;
+  p.tail_tiles = sp.tail_tiles;
+  p.split_s = sp.split_s;
+  p.slabs = a.slabs;
   cudaLaunchAttribute attr[2];
-  cudaLaunchConfig_t cfg = pair_config(dim3(2 * pairs), s, attr);
-  return (int)cudaLaunchKernelEx(&cfg, gemm_kernel, tmA, tmB, tmOut, tmU, tmL, p);
+  cudaLaunchConfig_t cfg = pair_config(dim3(2 * sp.pairs), s, attr);
+  cudaError_t e = sp.split_s > 1
+                      ? cudaLaunchKernelEx(&cfg, gemm_kernel<true>, tmA, tmB, tmOut, tmU, tmL, p)
+                      : cudaLaunchKernelEx(&cfg, gemm_kernel<false>, tmA, tmB, tmOut, tmU, tmL, p);
+  if (e != cudaSuccess || sp.split_s == 1) return (int)e;
+  // the split tiles' partial sums, added in slab order
+  cudaLaunchConfig_t rc = {};
+  rc.gridDim = dim3((unsigned)(sp.tail_tiles * (2 * BM / kReduceRows)));
+  rc.blockDim = dim3(kReduceRows * (BN / 4));
+  rc.stream = s;
+  cudaLaunchAttribute rattr[1];
+  rattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  rattr[0].val.programmaticStreamSerializationAllowed = 1;
+  rc.attrs = rattr;
+  rc.numAttrs = 1;
+  const int num_m = (int)((a.M + 2 * BM - 1) / (2 * BM)), num_n = (int)((a.N + BN - 1) / BN);
+  return (int)cudaLaunchKernelEx(&rc, split_reduce_kernel, (const float*)a.slabs, p, num_m, num_n);
 }
 
 }  // namespace
@@ -1050,6 +1210,14 @@ int launch_gemm(const GemmArgs& a, cudaStream_t s, bool* unsupported) {
     return 0;
   }
   return launch_persistent(a, s);
+}
+
+int64_t gemm_split_slabs(int64_t M, int64_t N, int64_t K, int32_t epilogue) {
+  if (M < 1 || N < 1 || K < 64 || M > (int64_t)INT32_MAX / 2 || N > (int64_t)INT32_MAX / 2 ||
+      K > (int64_t)INT32_MAX / 2)
+    return 0;
+  const SplitPlan sp = plan_split(M, N, K, epilogue == 0, INT64_MAX);
+  return sp.split_s > 1 ? (int64_t)sp.tail_tiles * sp.split_s : 0;
 }
 
 }  // namespace nvfp4

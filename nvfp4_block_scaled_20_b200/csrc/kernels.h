@@ -94,7 +94,14 @@ struct GemmArgs {
   int64_t ldu, ldl, rank;
   float lora_scale;
   void* u_scaled;
+  // Partial-sum slabs for splitting the last round's tiles along K (null or
+  // slab_cap 0: no split): slab_cap fp32 [256, 256] slabs, 16-byte aligned.
+  float* slabs;
+  int64_t slab_cap;
 };
+// Partial-sum slabs the launch of this GEMM would use with room for all of
+// them (0: it runs unsplit).
+int64_t gemm_split_slabs(int64_t M, int64_t N, int64_t K, int32_t epilogue);
 
 // Default bound of a GEMM pipeline wait, and the process-wide settings
 // (nvfp4_set_wait_limit, 0 restores the default; nvfp4_set_test_stall).

@@ -8,7 +8,7 @@ import torch
 
 import oracle
 import nvfp4_block_scaled_20_b200 as nv
-from nvfp4_block_scaled_20_b200 import synth
+from nvfp4_block_scaled_20_b200 import capi, synth
 from gpu_helpers import (DEV, assert_q_equal, gemm_tolerance, oracle_gemm_ref, require_gpu,
                          to_oracle)
 
@@ -284,3 +284,59 @@ def test_gemm_lora_host_validation():
     assert capi.nvfp4_gemm_lora(*args(128, 128, float("inf"), p)) == 1
     assert capi.nvfp4_gemm_lora(*args(128, 128, 1.0, p + 8)) == 3  # scratch misaligned
     assert capi.nvfp4_lora_scratch_bytes(2640, 128) == 2640 * 128 * 4
+
+
+def _split_case(M, N, K, seed):
+    x = synth.activation(seed, 1, M, K)
+    w = synth.activation(seed, 2, N, K)
+    aref = oracle.quantize_1d(to_oracle(x), sf_layout=oracle.SF_TCGEN05)
+    bref = oracle.quantize_1d(to_oracle(w), sf_layout=oracle.SF_TCGEN05)
+    return aref, bref, upload(aref, M, K), upload(bref, N, K)
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 512, 8192), (200, 400, 8192)])
+def test_split_k_when_tiles_are_fewer_than_pairs(M, N, K):
+    """A workspace with partial-sum slabs and fewer tiles than SM pairs: every
+    tile is cut along K into ranges of at least eight stages, the ranges'
+    fp32 sums added in slab order by the reduction kernel.  Both output types
+    within the GEMM bound of the oracle everywhere (ragged M and N included),
+    the same bits on a repeat, and the unsplit launch (error-word workspace)
+    within the bound too."""
+    assert capi.nvfp4_gemm_workspace_bytes(M, N, K, 0) > capi.nvfp4_workspace_bytes(0)
+    aref, bref, qa, qb = _split_case(M, N, K, 31)
+    y, s = oracle_gemm_ref(aref, bref, M, N, K)
+    for dt in (torch.float32, torch.bfloat16):
+        ws = nv.gemm_workspace(M, N, K)
+        o1 = nv.gemm(qa, qb, out_dtype=dt, ws=ws)
+        o2 = nv.gemm(qa, qb, out_dtype=dt, ws=ws)
+        plain = nv.gemm(qa, qb, out_dtype=dt, ws=nv.workspace(0))
+        torch.cuda.synchronize()
+        assert nv.device_error(ws) == 0
+        assert torch.equal(o1, o2)
+        tol = gemm_tolerance(y, s, dt == torch.bfloat16)
+        for got in (o1, plain):
+            err = np.abs(got.float().cpu().numpy().astype(np.float64) - y)
+            assert (err <= tol).all(), (dt, float((err / np.maximum(tol, 1e-30)).max()))
+
+
+def test_split_k_of_the_last_partial_round():
+    """One tile more than a round of SM pairs (15 x 5 tiles of 256 x 256): the
+    first round's tiles run whole and the last one is split along K among the
+    idle pairs.  Sampled outputs in every 256 x 256 tile (eight rows and
+    eight columns of each tile band, corners included) within the GEMM bound
+    of the oracle, whichever tile the schedule left for the last round."""
+    M, N, K = 15 * 256, 5 * 256, 8192
+    aref, bref, qa, qb = _split_case(M, N, K, 32)
+    ws = nv.gemm_workspace(M, N, K)
+    out = nv.gemm(qa, qb, out_dtype=torch.float32, ws=ws)
+    torch.cuda.synchronize()
+    assert nv.device_error(ws) == 0
+    rng = np.random.default_rng(5)
+    mi = np.unique(np.concatenate([t * 256 + np.r_[0, 255, rng.integers(0, 256, 6)]
+                                   for t in range(M // 256)]))
+    ni = np.unique(np.concatenate([t * 256 + np.r_[0, 255, rng.integers(0, 256, 6)]
+                                   for t in range(N // 256)]))
+    gm, gn = np.meshgrid(mi, ni, indexing="ij")
+    y, s = oracle_gemm_ref(aref, bref, M, N, K, gm.ravel(), gn.ravel())
+    got = out.cpu().numpy()[gm.ravel(), gn.ravel()].astype(np.float64)
+    assert (np.abs(got - y) <= gemm_tolerance(y, s, False)).all()
