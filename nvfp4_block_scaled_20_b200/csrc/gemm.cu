@@ -31,9 +31,9 @@
 //                groups' scales; B scales for all 256 tile columns in each
 //                CTA).  Keeping scale copies out of the MMA thread's in-order
 //                tcgen05 queue lets the MMAs run back to back.
-// Tensor memory (each CTA): accumulator 0 at columns [0, 256), accumulator 1
-// at [160, 416) -- the two share 96 columns, which the epilogue drains first
-// and releases -- and the two scale slots at [416, 512).
+// Tensor memory (each CTA): the two scale slots at columns [0, 96),
+// accumulator 0 at [96, 352) and accumulator 1 at [256, 512) -- the two share
+// 96 columns, which the epilogue drains first and releases.
 // Every wait is bounded (wall clock through %globaltimer); on a timeout the
 // CTA records NVFP4_ERR_TIMEOUT in the device error word, drains what it
 // issued and frees its tensor memory before returning.
@@ -69,9 +69,10 @@ constexpr int kSmemBytes =
     kStages * kStageBytes + kEpiStageBytes + 1024 /*align*/ + 512 /*barriers*/;
 // tensor memory columns
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAcc1Col = 160;   // accumulator 0 at column 0, 1 at 160
-constexpr uint32_t kOvlCols = 96;    // columns [160, 256) belong to both
-constexpr uint32_t kSfSlotCol = 416; // two scale slots of 48 columns
+constexpr uint32_t kSfSlotCol = 0;   // two scale slots of 48 columns
+constexpr uint32_t kAcc0Col = 96;    // accumulator 0 at column 96, 1 at 256
+constexpr uint32_t kAcc1Col = 256;
+constexpr uint32_t kOvlCols = 96;    // columns [256, 352) belong to both
 constexpr uint32_t kSfSlotCols = 48; // A: 4 per MMA k-block (16), B: 8 per k-block (32)
 constexpr int kSfSlots = 2;
 constexpr int kGroupM = 8;           // tile raster: 8 M-tiles per group
@@ -683,7 +684,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t t_acc = tmem + (b ? kAcc1Col : 0u);
+        const uint32_t t_acc = tmem + (b ? kAcc1Col : kAcc0Col);
         for (int kt = w.kt0; kt < w.kt1; ++kt, ++it) {
           if (!mbar_wait(smem_u32(&full[st]), st_ph, abort_flag, p.wait_limit_ns) ||
               !mbar_wait(smem_u32(&sf_full[slot]), slot_ph, abort_flag, p.wait_limit_ns)) {
@@ -755,7 +756,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t t_acc = tmem + (b ? kAcc1Col : 0u) + ((uint32_t)(quad * 32) << 16);
+      const uint32_t t_acc = tmem + (b ? kAcc1Col : kAcc0Col) + ((uint32_t)(quad * 32) << 16);
       const bool quad_live = m0 + quad * 32 < p.M;  // warp-uniform
       // The columns shared with the other accumulator (tile columns 160..255
       // of accumulator 0, 0..95 of accumulator 1) go first, split between
