@@ -51,8 +51,8 @@ TRAFFIC = {
     # wgrad_step, the first rep's six launches (after the four setup ones);
     # "gemm" is the GEMM with its split last round plus the reduction of the
     # split tiles' partial sums (gemm_kernel<true> + split_reduce_kernel)
-    "gemm": {"bytes_per_launch": 889843200 + 158941696 + 18881536 + 0,
-             "source_sha256": "d726cc240ca8c9a4404f585d01cabf1b1364170138dbb3a8f3c1e10376b6a5de"},
+    "gemm": {"bytes_per_launch": 978168832 + 162859776 + 18881280 + 0,
+             "source_sha256": "43178c1bc4b8648ddd91a3229f0b240e8bd59d53c7b01dc189ed4c72c88bcdf2"},
     "encode_x": {"bytes_per_launch": 954204160 + 251442176,
                  "source_sha256": "d443ba1bae7321cd2d15be6d2775c8c68c4ae04fb60685defd54ee1f4596e1ec"},
     "amax_x": {"bytes_per_launch": 939580928 + 470272,
