@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from conftest import ROOT
 from nvfp4_block_scaled_20_b200 import build, capi
@@ -43,6 +44,15 @@ def test_size_helpers(lib):
     assert capi.nvfp4_scales_bytes(64, 80, capi.NVFP4_SF_TCGEN05) == 128 * 8
     assert capi.nvfp4_workspace_bytes(0) >= 4
     assert capi.nvfp4_workspace_bytes(60) >= capi.nvfp4_workspace_bytes(0) + 240
+    # the GEMM's split-capable workspace is never below the plain one (the
+    # error word, plus one amax slot set with NVFP4_EPI_AMAX); without a
+    # device the launch would not split, so it is exactly the plain size
+    for M, N, K, epi in [(3072, 14336, 32768, 0), (64, 16, 64, 0), (8192, 14336, 3072, 17)]:
+        got = capi.nvfp4_gemm_workspace_bytes(M, N, K, epi)
+        plain = capi.nvfp4_workspace_bytes(1 if epi & capi.NVFP4_EPI_AMAX else 0)
+        assert got >= plain
+        if not torch.cuda.is_available():
+            assert got == plain
 
 
 def test_status_strings(lib):
