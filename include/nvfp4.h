@@ -349,7 +349,9 @@ NVFP4_API nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf,
  * this shape and epilogue (room for the error word, the amax partials and
  * one fp32 256 x 256 slab per split unit); nvfp4_workspace_bytes of the call
  * when the launch would not split.  Depends on the current device's SM
- * count; without a usable device, nvfp4_workspace_bytes of the call. */
+ * count; without a usable device, nvfp4_workspace_bytes of the call.  Like
+ * every workspace it serves one call in flight at a time (the split tiles'
+ * partial sums live in it until the call's reduction kernel has run). */
 NVFP4_API size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int32_t epilogue);
 
 /* Bytes of the scratch nvfp4_gemm_lora needs for an M-row activation and a
