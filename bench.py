@@ -52,7 +52,7 @@ TRAFFIC = {
     # "gemm" is the GEMM with its split last round plus the reduction of the
     # split tiles' partial sums (gemm_kernel<true> + split_reduce_kernel)
     "gemm": {"bytes_per_launch": 978168832 + 162859776 + 18881280 + 0,
-             "source_sha256": "43178c1bc4b8648ddd91a3229f0b240e8bd59d53c7b01dc189ed4c72c88bcdf2"},
+             "source_sha256": "a98bdb93b5a01ecee19b2418a8fcee018491071c9762879bac0daebc5c0ccf57"},
     "encode_x": {"bytes_per_launch": 954204160 + 251442176,
                  "source_sha256": "d443ba1bae7321cd2d15be6d2775c8c68c4ae04fb60685defd54ee1f4596e1ec"},
     "amax_x": {"bytes_per_launch": 939580928 + 470272,

@@ -34,6 +34,10 @@
 // Tensor memory (each CTA): the two scale slots at columns [0, 96),
 // accumulator 0 at [96, 352) and accumulator 1 at [256, 512) -- the two share
 // 96 columns, which the epilogue drains first and releases.
+// Given workspace slabs, the tiles left for the schedule's last, partial
+// round are cut along K into work units for the pairs that would idle; their
+// fp32 partial tiles go to the slabs and split_reduce_kernel, launched next on
+// the same stream, adds them in a fixed order and stores the output.
 // Every wait is bounded (wall clock through %globaltimer); on a timeout the
 // CTA records NVFP4_ERR_TIMEOUT in the device error word, drains what it
 // issued and frees its tensor memory before returning.
